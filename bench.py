@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark of one Medusa draft-and-verify step on B200.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+md_medusa_heads (K heads + per-head top-k) -> md_tree_build -> md_tree_attention
+(one layer of the verification pass) -> md_tree_accept. The default workload is
+the Llama-3.3-70B-shaped one at B = 1 (d 8192, V 128256, K 4, 64-candidate tree
+from top-10 heads, 64 q / 8 kv heads, dh 128, KV prefix 4096, greedy).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl medusa|reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs its own
+replica on its own GPU (requests are independent: no collective on the data
+path); the timed region is bracketed by barriers and the slowest rank's time
+is used; `value` counts the steps of all ranks.
+
+`--impl reference` times the CPU oracle (plain fp64 numpy, host cores) on a
+bounded sample of the same workload: the vocabulary projection and the
+residual block on a fraction of their output columns and the attention on the
+same fraction of its rows, scaled back to a whole step; tree build and
+acceptance run in full.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from seeded_inputs import gen, synth  # noqa: E402
+from seeded_inputs.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "Medusa head+tree-verify steps/s at 70B shapes B=1; HBM GB/s vs B200 peak"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# --------------------------------------------------------------------------- #
+# Algorithmic byte and flop counts (what the method must move / compute).
+# --------------------------------------------------------------------------- #
+def heads_bytes(w):
+    weights = 2 * w.K * (w.d * w.d + w.d + w.d * w.V)
+    return weights + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax
+
+
+def attention_bytes(w, P):
+    kv = sum(2 * w.Hkv * (p + w.T) * w.dh * 2 for p in P)
+    return kv + w.B * w.T * w.Hq * w.dh * (2 + 4)
+
+
+def attention_flops(w, P):
+    return sum(4 * w.Hq * w.T * (p + w.T) * w.dh for p in P)
+
+
+def accept_bytes(w):
+    return w.B * w.T * w.V * 4
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- #
+# Clock sampling during the timed region.
+# --------------------------------------------------------------------------- #
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join("/tmp", f"medusa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] not in ("", "[N/A]"))}
+
+
+# --------------------------------------------------------------------------- #
+# The oracle on a bounded sample (cpu_baseline leg and --impl reference).
+# --------------------------------------------------------------------------- #
+class OracleSampler:
+    """Times the CPU oracle on a fraction `frac` of the step's column/row work
+    and scales it back to one whole step. Inputs are drawn on the host from
+    the same seeded generator."""
+
+    def __init__(self, w, frac: float, seed_offset: int = 0):
+        from oracle import tree as ot
+        self.w = w
+        self.frac = frac
+        s = w.seed + seed_offset
+        d, V, K = w.d, w.V, w.K
+        rng = np.random.default_rng(1234)
+        self.cols_o = np.sort(rng.choice(d, max(1, int(round(d * frac))), replace=False))
+        self.cols_v = np.sort(rng.choice(V, max(1, int(round(V * frac))), replace=False))
+        kw = [gen.stream_key(s, n) for n in ("W1", "Wv", "b1", "h")]
+        ii = np.arange(d, dtype=np.uint64)
+        # W1[k, i, o] and Wv[k, i, v] at the sampled columns only (counter-based draws)
+        self.W1 = np.stack([gen.normal_bf16_at(kw[0], ((k * d + ii[:, None]) * d + self.cols_o[None, :]).astype(
+            np.uint64).ravel(), w.w_sigma).reshape(d, -1) for k in range(K)])
+        self.Wv = np.stack([gen.normal_bf16_at(kw[1], ((k * d + ii[:, None]) * V + self.cols_v[None, :]).astype(
+            np.uint64).ravel(), w.w_sigma).reshape(d, -1) for k in range(K)])
+        self.b1 = gen.normal_bf16(s, "b1", (K, d), w.w_sigma)
+        self.h = gen.normal_bf16(s, "h", (w.M, d), 1.0)
+        self.root = synth.root_tokens(s, w.B, V)
+        self.P = synth.prefix_lengths(s, w.B, *w.prefix)
+        tups = ot.select_tree(w.k_per_head, w.accept, w.n_nodes)
+        self.parent, self.rank, _ = ot.spec_from_tuples(tups)
+        self.q = gen.normal_bf16(s, "q", (w.B, w.T, w.Hq, w.dh), 1.0)
+        self.k = gen.normal_bf16(s, "k_cache", (w.B, w.Hkv, w.S_max, w.dh), 1.0)
+        self.v = gen.normal_bf16(s, "v_cache", (w.B, w.Hkv, w.S_max, w.dh), 1.0)
+        nrows = w.B * w.T * w.Hq
+        pick = rng.choice(nrows, max(1, int(round(nrows * frac))), replace=False)
+        self.rows = [(int(r // (w.T * w.Hq)), int((r // w.Hq) % w.T), int(r % w.Hq)) for r in pick]
+        self.topk_ids = rng.integers(0, V, (w.M, K, w.kmax)).astype(np.int32)
+        # z of the right shape for the sampled projection (its values do not change the work)
+        self.z = np.repeat(self.h[:, None, :], K, axis=1)
+        tokens = synth.synthetic_tree_tokens(s, w.B, self.parent, V, root_tokens=self.root)
+        self.tokens = tokens
+        self.logits = synth.planted_logits(s, self.parent, tokens, V, w.accept, sigma=w.logit_sigma, bump=w.bump)
+
+    def step(self):
+        """Returns the estimated seconds of one whole oracle step."""
+        from oracle import accept as oacc
+        from oracle import attention as oa
+        from oracle import heads as oh
+        from oracle import tree as ot
+        w = self.w
+        t0 = time.perf_counter()
+        oh.residual_block_columns(self.h, self.W1, self.b1[:, self.cols_o], self.cols_o)
+        t1 = time.perf_counter()
+        logits = oh.vocab_logits(self.z, self.Wv)          # self.Wv holds the sampled columns only
+        oh.heads_topk(logits, w.k_per_head, w.kmax)
+        t2 = time.perf_counter()
+        ot.tree_build(self.parent, self.rank, self.topk_ids, self.root, self.P)
+        t3 = time.perf_counter()
+        oa.tree_attention(self.q, self.k, self.v, self.P, self.parent, rows=self.rows)
+        t4 = time.perf_counter()
+        if w.mode == "greedy":
+            oacc.greedy_accept(self.logits, self.tokens, self.parent, w.K)
+        else:
+            oacc.typical_accept(self.logits, self.tokens, self.parent, w.K, w.temperature, w.eps, w.alpha)
+        t5 = time.perf_counter()
+        return (t1 - t0) / self.frac + (t2 - t1) / self.frac + (t3 - t2) + (t4 - t3) / self.frac + (t5 - t4)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    """--impl reference: the CPU oracle, K sample steps after W warm-ups."""
+    frac = args.ref_frac
+    smp = OracleSampler(w, frac)
+    for _ in range(args.warmup):
+        smp.step()
+    est = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        est.append(smp.step())
+    wall = time.perf_counter() - t0
+    sec = float(np.mean(est))
+    value = 1.0 / sec
+    sample = (f"per step: residual block and vocabulary projection on {frac:.4g} of their output columns, "
+              f"attention on {frac:.4g} of its (token, head) rows, scaled by 1/{frac:.4g}; tree build and "
+              f"acceptance in full; {args.steps} sample steps took {wall:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sec, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, None),
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, P):
+    return {"workload": w.name, "B": w.B, "heads_rows": w.M, "d": w.d, "V": w.V, "K": w.K,
+            "k_per_head": list(w.k_per_head), "tree_nodes": w.n_nodes, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+            "dh": w.dh, "prefix": list(w.prefix) if P is None else [int(p) for p in P], "accept": w.mode,
+            "l2": "inputs larger than L2: 8.99 GB of head weights stream every step; attention and acceptance "
+                  "inputs rotate over buffer sets totalling more than 2x L2"}
+
+
+# --------------------------------------------------------------------------- #
+# The CUDA arm.
+# --------------------------------------------------------------------------- #
+def run_medusa(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import medusa_draft_heads_b200 as md
+    from medusa_draft_heads_b200.step import MedusaStep
+    from seeded_inputs import device as sdev
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    seed = w.seed + rank
+    stream = torch.cuda.Stream(dev)
+
+    # ---- resident inputs -------------------------------------------------
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    W1 = sdev.fill_normal(torch.empty((w.K, w.d, w.d), **bf), seed, "W1", w.w_sigma)
+    b1 = sdev.fill_normal(torch.empty((w.K, w.d), **bf), seed, "b1", w.w_sigma)
+    Wv = sdev.fill_normal(torch.empty((w.K, w.d, w.V), **bf), seed, "Wv", w.w_sigma)
+    h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), seed, "h", 1.0)
+    root = torch.from_numpy(synth.root_tokens(seed, w.B, w.V)).to(dev)
+    P = synth.prefix_lengths(seed, w.B, *w.prefix)
+    prefix = torch.from_numpy(P).to(dev)
+    tups = md.select_tree(w.k_per_head, w.accept, w.n_nodes)
+    step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
+                      Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
+                      alpha=w.alpha, device=dev)
+    head_row = None
+    if w.M != w.B:
+        head_row = torch.arange(w.B, dtype=torch.int32, device=dev) * w.T
+
+    # attention / acceptance inputs: buffer sets that together exceed 2x L2
+    set_bytes = 2 * w.B * w.Hkv * w.S_max * w.dh * 2 + w.B * w.T * w.V * 4 + w.B * w.T * w.Hq * w.dh * 2
+    nsets = max(2, -(-2 * L2_BYTES // set_bytes))
+    with torch.cuda.stream(stream):
+        step.heads(h, W1, b1, Wv)
+        step.build(root, prefix, head_row)
+    stream.synchronize()
+    tokens = step.tokens.cpu().numpy()
+    parent_np = np.array(step.tree.parent)
+    logits_host = synth.planted_logits(seed, parent_np, tokens, w.V, w.accept, sigma=w.logit_sigma, bump=w.bump)
+    sets = []
+    for i in range(nsets):
+        q = sdev.fill_normal(torch.empty((w.B, w.T, w.Hq, w.dh), **bf), seed + 7919 * i, "q", 1.0)
+        kc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + 7919 * i, "k_cache", 1.0)
+        vc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + 7919 * i, "v_cache", 1.0)
+        lg = torch.from_numpy(logits_host).to(dev)
+        sets.append((q, kc, vc, lg))
+    torch.cuda.synchronize()
+
+    def one_step(i, ev=None):
+        q, kc, vc, lg = sets[i % nsets]
+        if ev is not None:
+            ev[0].record(stream)
+        step.heads(h, W1, b1, Wv)
+        if ev is not None:
+            ev[1].record(stream)
+        step.build(root, prefix, head_row)
+        if ev is not None:
+            ev[2].record(stream)
+        step.attention(q, kc, vc, prefix)
+        if ev is not None:
+            ev[3].record(stream)
+        step.accept(lg)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            one_step(i)
+    stream.synchronize()
+    status = md.device_status(stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        time.sleep(0.3)
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(args.steps):
+                one_step(i, evs[i])
+            end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = start.elapsed_time(end)
+    per_call = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+    clk = clocks.summary()
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * args.steps / (total_ms / 1000.0)
+
+    # ---- end to end through the public API with host buffers ---------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, dev, world, barrier)
+
+    if rank == 0:
+        peaks = measured_peaks()
+        hb = heads_bytes(w)
+        heads_ms = float(per_call[:, 0].mean())
+        achieved = hb / (heads_ms / 1000.0) / 1e9
+        ab = attention_bytes(w, P)
+        af = attention_flops(w, P)
+        attn_ms = float(per_call[:, 2].mean())
+        acc_ms = float(per_call[:, 3].mean())
+        step_bytes = hb + ab + accept_bytes(w)
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_baseline(w, args)
+        line = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, P),
+            "roofline": {"kernel": "md_medusa_heads (residual block + vocabulary stream + top-k merge)",
+                         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": args.traffic,
+                         "algorithmic_bytes": hb, "avg_ms": heads_ms, "peak_source": peaks["source"]},
+            "step_gbs": step_bytes / (ms_per_step / 1000.0) / 1e9 / 1.0,
+            "step_gbs_frac": step_bytes / (ms_per_step / 1000.0) / 1e9 / peaks["hbm_gbs"],
+            "per_call_ms": {"medusa_heads": heads_ms, "tree_build": float(per_call[:, 1].mean()),
+                            "tree_attention": attn_ms, "tree_accept": acc_ms},
+            "attention": {"bytes": ab, "flops": af, "gbs": ab / (attn_ms / 1000) / 1e9,
+                          "tflops": af / (attn_ms / 1000) / 1e12},
+            "accept": {"bytes": accept_bytes(w), "gbs": accept_bytes(w) / (acc_ms / 1000) / 1e9},
+            "gpu_launches": 8 * args.steps,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "accepted_len_mean": float(step.accept_len.float().mean().item()),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, dev, world, barrier):
+    """Same step through the public API, with this step's inputs copied from
+    pinned host memory and the result read back every step."""
+    import torch
+    q0, kc0, vc0, lg0 = sets[0]
+    Pn = prefix.cpu().numpy()
+    host = {
+        "h": h.cpu().pin_memory(), "root": root.cpu().pin_memory(), "prefix": prefix.cpu().pin_memory(),
+        "q": q0.cpu().pin_memory(),
+        "k_new": torch.stack([kc0[b, :, Pn[b]:Pn[b] + w.T].cpu() for b in range(w.B)]).pin_memory(),
+        "v_new": torch.stack([vc0[b, :, Pn[b]:Pn[b] + w.T].cpu() for b in range(w.B)]).pin_memory(),
+        "logits": lg0.cpu().pin_memory(),
+    }
+    out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
+                (("accept_len", step.accept_len), ("path", step.path), ("bonus", step.bonus))}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    steps = max(3, args.steps // 4)
+
+    def e2e_step():
+        h.copy_(host["h"], non_blocking=True)
+        root.copy_(host["root"], non_blocking=True)
+        prefix.copy_(host["prefix"], non_blocking=True)
+        q0.copy_(host["q"], non_blocking=True)
+        for b in range(w.B):
+            kc0[b, :, Pn[b]:Pn[b] + w.T].copy_(host["k_new"][b], non_blocking=True)
+            vc0[b, :, Pn[b]:Pn[b] + w.T].copy_(host["v_new"][b], non_blocking=True)
+        lg0.copy_(host["logits"], non_blocking=True)
+        step.run(h, W1, b1, Wv, root, prefix, q0, kc0, vc0, lg0, head_row=head_row)
+        out_host["accept_len"].copy_(step.accept_len, non_blocking=True)
+        out_host["path"].copy_(step.path, non_blocking=True)
+        out_host["bonus"].copy_(step.bonus, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = s.elapsed_time(e)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": world * steps / (ms / 1000.0), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "note": "per step: h, root token, prefix lengths, q, the tree tokens' K/V and the target logits "
+                    "copied in from pinned host memory; accept_len, path and bonus copied out; stream "
+                    "synchronised after every step"}
+
+
+def cpu_baseline(w, args):
+    frac = args.cpu_frac
+    smp = OracleSampler(w, frac)
+    smp.step()
+    est = []
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < args.cpu_seconds or len(est) < 2:
+        est.append(smp.step())
+    sec = float(np.median(est))
+    return {"value": 1.0 / sec, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(est)} oracle sample steps in {time.perf_counter() - t0:.1f} s; each: residual block "
+                      f"and vocabulary projection on {frac:.4g} of their output columns, attention on {frac:.4g} of "
+                      f"its (token, head) rows, scaled by 1/{frac:.4g}; tree build and acceptance in full"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["medusa", "reference"], default="medusa")
+    ap.add_argument("--workload", default="llama3-70b", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-frac", type=float, default=1 / 64)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-frac", type=float, default=1 / 512)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per heads call from an ncu capture of the current kernels")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args, w)
+        return
+    run_medusa(args, w)
+
+
+if __name__ == "__main__":
+    main()

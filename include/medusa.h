@@ -1,0 +1,253 @@
+/*
+ * medusa.h -- C ABI of libmedusa: the per-step Medusa draft-and-verify chain
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The step, as "Medusa heads versus separate draft model" describes it
+ * (sections "What each one is" and "Acceptance", tree paragraph):
+ *   1. K draft heads read the target's last hidden state once, in parallel;
+ *      head k is one residual block followed by its own vocabulary
+ *      projection and guesses the token k positions ahead;
+ *   2. the top few candidates of each head are combined into a tree;
+ *   3. the target verifies every branch in one pass with a tree attention
+ *      mask;
+ *   4. the step advances along the longest branch that matches.
+ * Calls: md_medusa_heads (1), md_tree_build (2), md_tree_attention (3, one
+ * attention layer of the verification pass), md_tree_accept (4).
+ *
+ * Conventions (all calls):
+ *  - Tensor pointers are DEVICE pointers unless a comment says "host". The
+ *    caller allocates and owns every buffer, including the workspace each
+ *    call asks for; the library keeps no pointer after a call returns.
+ *  - bf16 tensors are passed as uint16_t bit patterns (md_bf16).
+ *  - Layouts are dense row-major in the index order written in brackets.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream). Outputs are ready when the stream reaches the
+ *    call's point.
+ *  - Shapes and pointers are checked on the host first; on error the call
+ *    returns a negative md_status and launches nothing.
+ *  - Errors that depend on device data (a prefix that does not fit the KV
+ *    cache, a row or token id out of range) never trap: the kernels skip the
+ *    offending item, write a defined value (-1 ids, zeros) and set a bit in a
+ *    device status word read by md_get_device_status().
+ *  - No C++ exception crosses this interface.
+ *  - Kernels use no floating-point atomics: results are bitwise
+ *    reproducible run to run for the same inputs and sizes.
+ */
+#ifndef MEDUSA_H
+#define MEDUSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MD_API __attribute__((visibility("default")))
+#else
+#define MD_API
+#endif
+
+typedef int32_t md_status;
+typedef uint16_t md_bf16;
+
+enum {
+  MD_OK = 0,
+  MD_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, bad tree spec     */
+  MD_ERR_UNSUPPORTED = -2, /* valid but outside the supported ranges below      */
+  MD_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch, copy, ...)    */
+  MD_ERR_WORKSPACE = -4,   /* workspace pointer null or smaller than required   */
+  MD_ERR_TIMEOUT = -5      /* a bounded device wait gave up (device status bit) */
+};
+
+/* Bits of the device status word (md_get_device_status). */
+enum {
+  MD_DEV_BAD_PREFIX = 1,   /* prefix_len[b] < 0 or prefix_len[b] + T > S_max     */
+  MD_DEV_BAD_ROW = 2,      /* head_row[b] outside [0, M)                         */
+  MD_DEV_BAD_TOKEN = 4,    /* a token id outside [0, V) reached tree_accept      */
+  MD_DEV_TIMEOUT = 8       /* a pipeline wait exceeded its bound                 */
+};
+
+/* Supported ranges (anything else: MD_ERR_UNSUPPORTED).
+ *   heads:     1 <= K <= 8, 1 <= k_i <= kmax <= 16, d % 64 == 0, V % 8 == 0,
+ *              V >= 256, 1 <= M <= 8 on the streaming path.
+ *   tree:      1 <= T <= 128, depth <= K.
+ *   attention: dh in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16.
+ */
+#define MD_MAX_T 128
+#define MD_MAX_K 8
+#define MD_MAX_KMAX 16
+
+/* ------------------------------------------------------------------------ */
+/* Tree spec.                                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Opaque, host-only description of a fixed candidate tree. */
+typedef struct md_tree md_tree;
+
+/* Creates a tree spec.
+ * Source: "Medusa heads versus separate draft model", section "Acceptance",
+ * tree paragraph ("take the top few candidates from each head, form a tree
+ * of combinations").
+ *
+ * Node 0 is the root (the token the target already emitted). A node at
+ * depth k >= 1 is a candidate from head k: it holds head_rank[j], the rank
+ * of its token in head k's top-k list.
+ *
+ * parent     host [T]: parent[0] = -1; 0 <= parent[j] < j for j >= 1.
+ * head_rank  host [T]: head_rank[0] ignored; 0 <= head_rank[j] < k_per_head[depth(j)-1].
+ * T          nodes including the root, 1..MD_MAX_T.
+ * K          number of heads; every depth must be <= K.
+ * k_per_head host [K]: top-k of each head.
+ * out        receives a handle; free it with md_tree_destroy.
+ * Two children of one node must not share a rank (their tokens would be
+ * equal). The spec is copied; the arrays may be freed after the call.
+ * Allocates host memory only. Errors: MD_ERR_INVALID_ARG for any violation. */
+MD_API md_status md_tree_create(const int32_t* parent, const int32_t* head_rank, int32_t T, int32_t K,
+                         const int32_t* k_per_head, md_tree** out);
+MD_API md_status md_tree_destroy(md_tree* tree);
+/* T and the deepest depth of a tree (either pointer may be NULL). */
+MD_API md_status md_tree_info(const md_tree* tree, int32_t* T, int32_t* max_depth);
+
+/* ------------------------------------------------------------------------ */
+/* 1. Draft heads with fused per-head top-k.                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes md_medusa_heads needs for these sizes. */
+MD_API md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax, size_t* bytes);
+
+/* The K Medusa heads on M hidden rows, fused with a top-k per head.
+ * Source: "Medusa heads versus separate draft model", sections "What each
+ * one is" (one residual block and its own vocabulary projection per head,
+ * all heads on the same hidden state, run once in parallel) and "Cost per
+ * step" (block d x d + bias; projection d x V, no bias).
+ *
+ *   u[m,k,o]      = b1[k,o] + sum_i h[m,i] * W1[k,i,o]          (fp32 accumulate)
+ *   z[m,k,o]      = bf16_rne( h[m,o] + u / (1 + exp(-u)) )        (SiLU residual)
+ *   logit[m,k,v]  = sum_i z[m,k,i] * Wv[k,i,v]                   (fp32 accumulate)
+ *   topk_*[m,k,:] = the k_per_head[k] largest logits of row (m,k), ordered
+ *                   by (value descending, id ascending); slots past
+ *                   k_per_head[k] hold id -1 and value -inf.
+ *
+ * h          [M, d] bf16.        W1 [K, d, d] bf16 (input-major: W1[k][i][o]).
+ * b1         [K, d] bf16.        Wv [K, d, V] bf16 (input-major: Wv[k][i][v]).
+ * k_per_head host [K].           kmax: stride of the top-k outputs (>= every k_i).
+ * topk_ids   [M, K, kmax] int32, topk_vals [M, K, kmax] fp32 (outputs).
+ * logits_dbg [M, K, V] fp32 or NULL: when given, the full logits are also
+ *            written (debug / parity only; the fused path never needs them).
+ * ws, ws_bytes: workspace of at least md_heads_workspace() bytes.
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED, MD_ERR_WORKSPACE, MD_ERR_CUDA. */
+MD_API md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
+                          int32_t M, int32_t d, int32_t V, int32_t K, const int32_t* k_per_head,
+                          int32_t kmax, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 2. Candidate tree construction.                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Tokens, parents, ancestor mask and position ids of the tree for B requests.
+ * Source: "Medusa heads versus separate draft model", section "Acceptance",
+ * tree paragraph.
+ *
+ *   tokens[b,0] = root_token[b];
+ *   tokens[b,j] = topk_ids[row_b, depth(j)-1, head_rank[j]]  (j >= 1),
+ *                 row_b = head_row ? head_row[b] : b;
+ *   parent[j]   = the tree's parent array (root -1);
+ *   anc[j,w]    bit (i % 32) of word w = i / 32 is set iff node i is an
+ *               ancestor of j or j itself (W = ceil(T/32) words per node);
+ *   pos[b,j]    = prefix_len[b] + depth(j)   (position id for the target's
+ *               rotary embedding; the KV slot of node j is prefix_len[b] + j).
+ *
+ * topk_ids [M, K, kmax] int32 from md_medusa_heads.  head_row [B] int32 or NULL.
+ * root_token [B] int32.  prefix_len [B] int32.
+ * tokens [B, T] int32, parent [T] int32, anc [T, W] uint32, pos [B, T] int32.
+ * A head_row outside [0, M) sets MD_DEV_BAD_ROW and that request's candidate
+ * tokens are -1. Errors: MD_ERR_INVALID_ARG, MD_ERR_CUDA. */
+MD_API md_status md_tree_build(const md_tree* tree, const int32_t* topk_ids, int32_t M, int32_t kmax,
+                        const int32_t* head_row, const int32_t* root_token, const int32_t* prefix_len,
+                        int32_t B, int32_t* tokens, int32_t* parent, uint32_t* anc, int32_t* pos,
+                        void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 3. Tree-masked attention (one layer of the verification pass).            */
+/* ------------------------------------------------------------------------ */
+
+MD_API md_status md_attention_workspace(int32_t B, int32_t T, int32_t Hq, int32_t Hkv, int32_t dh,
+                                 int32_t S_max, size_t* bytes);
+
+/* Attention of the T tree tokens over the KV prefix plus the tree.
+ * Source: "Medusa heads versus separate draft model", section "Acceptance",
+ * tree paragraph ("verify all branches in one pass with a tree attention
+ * mask").
+ *
+ *   out[b,t,h,:] = sum_j softmax_j( scale * q[b,t,h,:] . K[b,g,j,:] ) V[b,g,j,:]
+ *   over key slots j in [0, P_b) and P_b + a for every ancestor a of t
+ *   (t included), with P_b = prefix_len[b] and KV head g = h / (Hq / Hkv).
+ *
+ * q       [B, T, Hq, dh] bf16 (already rotated by the caller).
+ * k_cache, v_cache [B, Hkv, S_max, dh] bf16; slots [P_b, P_b + T) hold the
+ *         tree tokens' own K/V (node j at slot P_b + j).
+ * prefix_len [B] int32; P_b + T > S_max or P_b < 0 sets MD_DEV_BAD_PREFIX
+ *         and writes zeros for that request.
+ * scale   softmax scale; 0 means 1/sqrt(dh).
+ * out     [B, T, Hq, dh] fp32.
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED, MD_ERR_WORKSPACE, MD_ERR_CUDA. */
+MD_API md_status md_tree_attention(const md_bf16* q, const md_bf16* k_cache, const md_bf16* v_cache,
+                            const int32_t* prefix_len, int32_t S_max, const md_tree* tree, int32_t B,
+                            int32_t Hq, int32_t Hkv, int32_t dh, float scale, float* out, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 4. Acceptance of the longest matching branch.                             */
+/* ------------------------------------------------------------------------ */
+
+enum { MD_ACCEPT_GREEDY = 0, MD_ACCEPT_TYPICAL = 1 };
+
+MD_API md_status md_accept_workspace(int32_t B, int32_t T, int32_t V, size_t* bytes);
+
+/* Longest accepted root-to-node path per request, and the bonus token.
+ * Source: "Medusa heads versus separate draft model", section "Acceptance",
+ * tree paragraph ("if any branch matches, the step advances along it"), and
+ * section "Training" (typical acceptance: accepts more drafts, not lossless).
+ *
+ * Row t of logits is the target's distribution for the token after node t.
+ * Non-root node j passes when
+ *   greedy : tokens[b,j] == argmax_v logits[b,parent(j),v]  (lowest id on ties)
+ *   typical: p(tokens[b,j]) > min(eps, alpha * exp(-H)), where p = softmax of
+ *            logits[b,parent(j),:] / temperature and H is its entropy (nats).
+ * A node is accepted when it and all its ancestors below the root pass.
+ * accept_len[b] = L, the deepest accepted depth (0..max depth);
+ * path[b, 0..L] = root .. the accepted depth-L node with the smallest index,
+ *                 path[b, L+1..K] = -1 (K = the heads, the tree's max depth);
+ * bonus[b]      = argmax of the last accepted node's row (lowest id on ties).
+ *
+ * logits [B, T, V] fp32.  tokens [B, T] int32 (from md_tree_build).
+ * K      width of `path` minus one (>= the tree's max depth).
+ * accept_len [B], path [B, K+1], bonus [B] int32 (outputs).
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED, MD_ERR_WORKSPACE, MD_ERR_CUDA. */
+MD_API md_status md_tree_accept(const float* logits, int32_t V, const int32_t* tokens, const md_tree* tree,
+                         int32_t B, int32_t K, int32_t mode, float temperature, float eps, float alpha,
+                         int32_t* accept_len, int32_t* path, int32_t* bonus, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Status.                                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Synchronises `stream`, then stores the device status word (MD_DEV_* bits
+ * set by kernels since the last clear) in *out; clears it if `clear` != 0. */
+MD_API md_status md_get_device_status(void* stream, int32_t* out, int32_t clear);
+
+/* Static description of a status code. */
+MD_API const char* md_status_string(md_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+MD_API int32_t md_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEDUSA_H */

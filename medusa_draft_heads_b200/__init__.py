@@ -1,0 +1,15 @@
+"""B200-native Medusa draft-and-verify step: four CUDA calls behind a C ABI.
+
+    medusa_heads   K draft heads (residual SiLU block + vocabulary projection)
+                   fused with a per-head top-k
+    tree_build     candidate tree: tokens, parents, ancestor bitsets, positions
+    tree_attention tree-masked GQA attention over the KV prefix plus the tree
+    tree_accept    longest accepted branch (greedy or typical) and bonus token
+
+The kernels live in ``libmedusa.so`` (built from ``csrc/`` for sm_100a); this
+package only marshals arguments to it.
+"""
+from .binding import (MedusaError, Tree, accept_workspace_bytes, attention_workspace_bytes,  # noqa: F401
+                      device_status, heads_workspace_bytes, lib, medusa_heads, tree_accept, tree_attention,
+                      tree_build, version, workspace)
+from .tree_spec import select_tree, tree_arrays  # noqa: F401

@@ -1,0 +1,211 @@
+// Acceptance of the longest matching branch.
+//
+// Source: "Medusa heads versus separate draft model", section "Acceptance",
+// tree paragraph (advance along the branch that matches), and section
+// "Training" (typical acceptance, which accepts more drafts under sampling and
+// is not lossless).
+//
+//   accept_rows_kernel  one pass over a chunk of one target-logit row: the
+//                       argmax (lowest id on ties) and, for the typical rule,
+//                       the online max m, S = sum e^(x-m), W = sum (x-m) e^(x-m)
+//                       of x = logits / temperature (HBM-bound, 16-byte loads)
+//   accept_walk_kernel  per request: merge the chunks, test every node against
+//                       its parent's row, propagate acceptance down the tree
+//                       level by level, pick the deepest accepted node (lowest
+//                       index on ties), emit its path and the bonus token.
+#pragma once
+
+#include "common.cuh"
+
+namespace md {
+namespace acc {
+
+constexpr int kRowThreads = 256;
+constexpr int kPartFloats = 8;  // best value, best id (bits), m, S, W, pad
+
+struct Args {
+  const float* logits;     // [B, T, V]
+  const int32_t* tokens;   // [B, T]
+  int32_t* accept_len;     // [B]
+  int32_t* path;           // [B, K + 1]
+  int32_t* bonus;          // [B]
+  float* part;             // [B * T, nchunks, 8]
+  int T, V, K, nchunks, chunk_len, mode;
+  float inv_temp, log_eps, log_alpha;
+};
+
+struct Soft {
+  float m, S, W;
+};
+
+// Combine two (max, sum e^(x-max), sum (x-max) e^(x-max)) summaries.
+__device__ __forceinline__ Soft soft_merge(Soft a, Soft b) {
+  if (a.S == 0.f) return b;
+  if (b.S == 0.f) return a;
+  const float m = fmaxf(a.m, b.m);
+  const float ea = expf(a.m - m), eb = expf(b.m - m);
+  Soft r;
+  r.m = m;
+  r.S = a.S * ea + b.S * eb;
+  r.W = ea * (a.W + (a.m - m) * a.S) + eb * (b.W + (b.m - m) * b.S);
+  return r;
+}
+
+__device__ __forceinline__ void soft_add(Soft& s, float y) {
+  if (s.S == 0.f) {
+    s.m = y;
+    s.S = 1.f;
+    s.W = 0.f;
+    return;
+  }
+  if (y > s.m) {
+    const float sc = expf(s.m - y);
+    s.W = sc * (s.W + (s.m - y) * s.S);
+    s.S *= sc;
+    s.m = y;
+  }
+  const float e = expf(y - s.m);
+  s.S += e;
+  s.W = fmaf(y - s.m, e, s.W);
+}
+
+__global__ void __launch_bounds__(kRowThreads) accept_rows_kernel(Args a) {
+  const int row = blockIdx.y, c = blockIdx.x;
+  const int v0 = c * a.chunk_len;
+  const int v1 = min(a.V, v0 + a.chunk_len);
+  const float* x = a.logits + size_t(row) * a.V;
+  float bv = -INFINITY;
+  int bi = INT_MAX;
+  Soft sm{-INFINITY, 0.f, 0.f};
+  const bool typical = a.mode == MD_ACCEPT_TYPICAL;
+  for (int v = v0 + threadIdx.x * 4; v < v1; v += kRowThreads * 4) {
+    const float4 f = ld_stream_f4(x + v);
+    const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (better(fv[e], v + e, bv, bi)) {
+        bv = fv[e];
+        bi = v + e;
+      }
+      if (typical) soft_add(sm, fv[e] * a.inv_temp);
+    }
+  }
+  // Block reduction (fixed shuffle tree, then warps in order).
+  __shared__ float sv[kRowThreads / 32];
+  __shared__ int si[kRowThreads / 32];
+  __shared__ Soft ss[kRowThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (better(ov, oi, bv, bi)) {
+      bv = ov;
+      bi = oi;
+    }
+    if (typical) {
+      Soft o;
+      o.m = __shfl_xor_sync(0xffffffffu, sm.m, off);
+      o.S = __shfl_xor_sync(0xffffffffu, sm.S, off);
+      o.W = __shfl_xor_sync(0xffffffffu, sm.W, off);
+      sm = (lane & off) ? soft_merge(o, sm) : soft_merge(sm, o);
+    }
+  }
+  if (lane == 0) {
+    sv[warp] = bv;
+    si[warp] = bi;
+    ss[warp] = sm;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kRowThreads / 32; ++w) {
+      if (better(sv[w], si[w], bv, bi)) {
+        bv = sv[w];
+        bi = si[w];
+      }
+      if (typical) sm = soft_merge(sm, ss[w]);
+    }
+    float* p = a.part + (size_t(row) * a.nchunks + c) * kPartFloats;
+    p[0] = bv;
+    p[1] = __int_as_float(bi);
+    p[2] = sm.m;
+    p[3] = sm.S;
+    p[4] = sm.W;
+  }
+}
+
+__global__ void __launch_bounds__(MD_MAX_T) accept_walk_kernel(const __grid_constant__ TreeParams tp, Args a) {
+  const int b = blockIdx.x;
+  const int j = threadIdx.x;
+  const int T = tp.T;
+  __shared__ int amax[MD_MAX_T];
+  __shared__ float mrow[MD_MAX_T], logS[MD_MAX_T], Hrow[MD_MAX_T];
+  __shared__ int accd[MD_MAX_T];
+  __shared__ int wkey[MD_MAX_T / 32];
+  const bool typical = a.mode == MD_ACCEPT_TYPICAL;
+
+  if (j < T) {
+    const float* p = a.part + size_t(b * T + j) * a.nchunks * kPartFloats;
+    float bv = p[0];
+    int bi = __float_as_int(p[1]);
+    Soft sm{p[2], p[3], p[4]};
+    for (int c = 1; c < a.nchunks; ++c) {
+      const float* q = p + size_t(c) * kPartFloats;
+      const int qi = __float_as_int(q[1]);
+      if (better(q[0], qi, bv, bi)) {
+        bv = q[0];
+        bi = qi;
+      }
+      if (typical) sm = soft_merge(sm, Soft{q[2], q[3], q[4]});
+    }
+    amax[j] = bi;
+    if (typical) {
+      mrow[j] = sm.m;
+      logS[j] = logf(sm.S);
+      Hrow[j] = logS[j] - sm.W / sm.S;
+    }
+  }
+  __syncthreads();
+  bool match = false;
+  if (j > 0 && j < T) {
+    const int par = tp.parent[j];
+    const int tok = a.tokens[size_t(b) * T + j];
+    if (!typical) {
+      match = tok == amax[par];
+    } else if (tok >= 0 && tok < a.V) {
+      const float y = a.logits[(size_t(b) * T + par) * a.V + tok] * a.inv_temp;
+      const float logp = y - mrow[par] - logS[par];
+      match = logp > fminf(a.log_eps, a.log_alpha - Hrow[par]);
+    } else {
+      set_status(MD_DEV_BAD_TOKEN);
+    }
+  }
+  if (j < MD_MAX_T) accd[j] = (j == 0) ? 1 : 0;
+  __syncthreads();
+  for (int level = 1; level <= tp.max_depth; ++level) {
+    if (j < T && tp.depth[j] == level) accd[j] = match && accd[tp.parent[j]];
+    __syncthreads();
+  }
+  // Deepest accepted node, lowest index on ties: max of depth*256 + (255 - j).
+  int key = (j < T && accd[j]) ? (tp.depth[j] << 8) | (255 - j) : -1;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, off));
+  if ((j & 31) == 0) wkey[j >> 5] = key;
+  __syncthreads();
+  if (j == 0) {
+    for (int w = 1; w < MD_MAX_T / 32; ++w) key = max(key, wkey[w]);
+    const int L = key >> 8;
+    int node = 255 - (key & 255);
+    a.accept_len[b] = L;
+    a.bonus[b] = amax[node];
+    int32_t* pp = a.path + size_t(b) * (a.K + 1);
+    for (int i = a.K; i > L; --i) pp[i] = -1;
+    for (int i = L; i >= 0; --i) {
+      pp[i] = node;
+      node = tp.parent[node];
+    }
+  }
+}
+
+}  // namespace acc
+}  // namespace md

@@ -1,0 +1,496 @@
+// Medusa draft heads with a fused per-head top-k, small-M streaming path.
+//
+// Source: "Medusa heads versus separate draft model", sections "What each one
+// is" and "Cost per step": head k = one residual block (d x d + bias) and its
+// own d x V vocabulary projection (no bias), all heads on the same hidden
+// state, once per step. At small batch the heads are bound by the bytes of
+// their weights (8.94 GB for four heads at d = 8,192, V = 128,256), so both
+// phases stream the weights once from HBM with 16-byte or TMA loads and do the
+// arithmetic in fp32 on the CUDA cores.
+//
+//   phase 1  heads_w1_kernel       u = h W1_k + b1_k, z_k = bf16(h + SiLU(u))
+//   phase 2  heads_vocab_kernel    logits tile = z_k Wv_k[:, tile] and its top-k
+//   phase 3  heads_merge_kernel    top-k over every tile's candidates
+#pragma once
+
+#include "common.cuh"
+
+namespace md {
+namespace heads {
+
+constexpr int kTileV = 256;         // vocabulary columns of one phase-2 work unit
+constexpr int kStageRows = 64;      // hidden rows per TMA stage
+constexpr int kConsumerWarps = 8;   // phase-2 math warps (one more warp feeds TMA)
+constexpr int kZPad = 8;            // z row i is stored as 8 bf16 (one per m), 16 B
+constexpr int kW1Threads = 256;
+constexpr int kW1TileO = 256;       // phase-1 output columns per CTA
+constexpr int kW1MaxRows = 1024;    // phase-1 hidden rows per CTA (split-K)
+constexpr int kMaxM = 8;
+constexpr uint32_t kStageWBytes = kStageRows * kTileV * 2;  // 32 KB
+constexpr uint32_t kStageZBytes = kStageRows * kZPad * 2;   // 1 KB
+constexpr int kSmemBudget = 227 * 1024;
+
+struct Plan {
+  int M, d, V, K, kmax;
+  int ntile_o;  // phase-1 column tiles
+  int splits;   // phase-1 split-K factor
+  int rows;     // phase-1 rows per split
+  int ntiles;   // phase-2 vocabulary tiles
+  int units;    // K * ntiles
+  int nstages;  // phase-2 pipeline depth
+  size_t off_zt, off_part, off_cnt, off_cval, off_cid, bytes;
+};
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+inline int vocab_smem_bytes(int M, int nstages) {
+  // stages + mbarriers + cross-warp reduction + reduced logits + 1 KB alignment slack
+  return nstages * int(kStageWBytes + kStageZBytes) + 2 * nstages * 8 + kConsumerWarps * M * kTileV * 4 +
+         M * kTileV * 4 + 1024 + 64;
+}
+
+inline Plan make_plan(int M, int d, int V, int K, int kmax, int num_sms) {
+  Plan p{};
+  p.M = M; p.d = d; p.V = V; p.K = K; p.kmax = kmax;
+  p.ntile_o = (d + kW1TileO - 1) / kW1TileO;
+  int splits = 1;
+  while (d / splits > kW1MaxRows) splits *= 2;
+  while (p.ntile_o * K * splits < 4 * num_sms && d / (splits * 2) >= 64 && (d / (splits * 2)) % 8 == 0) splits *= 2;
+  p.splits = splits;
+  p.rows = d / splits;
+  p.ntiles = (V + kTileV - 1) / kTileV;
+  p.units = K * p.ntiles;
+  int ns = 8;
+  while (ns > 2 && vocab_smem_bytes(M, ns) > kSmemBudget) --ns;
+  p.nstages = ns;
+  size_t o = 0;
+  p.off_zt = o;   o = align256(o + size_t(K) * d * kZPad * 2);
+  p.off_part = o; o = align256(o + size_t(splits) * K * M * d * 4);
+  p.off_cnt = o;  o = align256(o + size_t(K) * p.ntile_o * 4);
+  p.off_cval = o; o = align256(o + size_t(M) * K * p.ntiles * kmax * 4);
+  p.off_cid = o;  o = align256(o + size_t(M) * K * p.ntiles * kmax * 4);
+  p.bytes = o;
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// Phase 1: residual block, split over hidden rows, deterministic finish.
+// grid (ntile_o, splits, K), 256 threads. Each warp owns rows w, w+8, ...
+// of the split, each lane 8 output columns; partial sums go to `part`, and
+// the last CTA of a (head, column tile) sums the splits in order and applies
+// bias, SiLU and the residual.
+// ---------------------------------------------------------------------------
+struct W1Args {
+  const uint16_t* h;   // [M, d]
+  const uint16_t* W1;  // [K, d, d]
+  const uint16_t* b1;  // [K, d]
+  uint16_t* zt;        // [K, d, 8]
+  float* part;         // [splits, K, M, d]
+  int* counters;       // [K, ntile_o]
+  int d, K, splits, rows, ntile_o;
+};
+
+template <int M>
+__global__ void __launch_bounds__(kW1Threads) heads_w1_kernel(W1Args a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint4* hs = reinterpret_cast<uint4*>(smem);                          // [rows] x 8 bf16
+  float* red = reinterpret_cast<float*>(smem + size_t(a.rows) * 16);   // [8 warps][M][256]
+  __shared__ int is_last;
+
+  pdl_launch_dependents();
+
+  const int k = blockIdx.z, s = blockIdx.y, ct = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = a.d;
+  const int i0 = s * a.rows;
+  const int o = ct * kW1TileO + lane * 8;
+  const bool col_ok = o < d;
+
+  for (int r = threadIdx.x; r < a.rows; r += kW1Threads) {
+    uint16_t v[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) v[m] = (m < M) ? a.h[size_t(m) * d + i0 + r] : uint16_t(0);
+    hs[r] = make_uint4(v[0] | (uint32_t(v[1]) << 16), v[2] | (uint32_t(v[3]) << 16), v[4] | (uint32_t(v[5]) << 16),
+                       v[6] | (uint32_t(v[7]) << 16));
+  }
+  __syncthreads();
+
+  float acc[M][8];
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[m][c] = 0.f;
+
+  if (col_ok) {
+    const uint16_t* wrow = a.W1 + (size_t(k) * d + i0) * d + o;
+    constexpr int U = 4;
+    int r = warp;
+    for (; r + (U - 1) * kConsumerWarps < a.rows; r += U * kConsumerWarps) {
+      uint4 w[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) w[u] = ld_stream_v4(wrow + size_t(r + u * kConsumerWarps) * d);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint4 hv = hs[r + u * kConsumerWarps];
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float hm = (m & 1) ? bf16hi(hw[m >> 1]) : bf16lo(hw[m >> 1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            acc[m][2 * c] = fmaf(hm, bf16lo(ww[c]), acc[m][2 * c]);
+            acc[m][2 * c + 1] = fmaf(hm, bf16hi(ww[c]), acc[m][2 * c + 1]);
+          }
+        }
+      }
+    }
+    for (; r < a.rows; r += kConsumerWarps) {
+      const uint4 w = ld_stream_v4(wrow + size_t(r) * d);
+      const uint4 hv = hs[r];
+      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const float hm = (m & 1) ? bf16hi(hw[m >> 1]) : bf16lo(hw[m >> 1]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[m][2 * c] = fmaf(hm, bf16lo(ww[c]), acc[m][2 * c]);
+          acc[m][2 * c + 1] = fmaf(hm, bf16hi(ww[c]), acc[m][2 * c + 1]);
+        }
+      }
+    }
+  }
+
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    float4* dst = reinterpret_cast<float4*>(red + (size_t(warp) * M + m) * kW1TileO + lane * 8);
+    dst[0] = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+    dst[1] = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
+  }
+  __syncthreads();
+
+  const int t = threadIdx.x;
+  const int col = ct * kW1TileO + t;
+  if (col < d) {
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) v += red[(size_t(w) * M + m) * kW1TileO + t];
+      a.part[((size_t(s) * a.K + k) * M + m) * d + col] = v;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (t == 0) {
+    const int ticket = atomicAdd(&a.counters[k * a.ntile_o + ct], 1);
+    is_last = (ticket == a.splits - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (col < d) {
+    const float bias = bf16_to_f32(a.b1[size_t(k) * d + col]);
+    uint16_t zv[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      if (m < M) {
+        float u = 0.f;
+        for (int sp = 0; sp < a.splits; ++sp) u += __ldcg(&a.part[((size_t(sp) * a.K + k) * M + m) * d + col]);
+        u += bias;
+        const float hval = bf16_to_f32(a.h[size_t(m) * d + col]);
+        zv[m] = f32_to_bf16_rne(hval + u / (1.0f + expf(-u)));
+      } else {
+        zv[m] = 0;
+      }
+    }
+    reinterpret_cast<uint4*>(a.zt)[size_t(k) * d + col] =
+        make_uint4(zv[0] | (uint32_t(zv[1]) << 16), zv[2] | (uint32_t(zv[3]) << 16), zv[4] | (uint32_t(zv[5]) << 16),
+                   zv[6] | (uint32_t(zv[7]) << 16));
+  }
+  if (t == 0) a.counters[k * a.ntile_o + ct] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Phase 2: persistent vocabulary stream with the per-tile top-k fused in.
+// grid = min(#SMs, K * ntiles), 288 threads: warps 0..7 do the math, warp 8
+// issues the TMA loads. A work unit is (head k, 256-column tile); it walks
+// d / 64 stages of [64 rows x 256 cols] of Wv_k plus the matching 64 rows of
+// z_k. Warp w multiplies rows 8w..8w+7 of each stage, lane l columns
+// 8l..8l+7, fp32 accumulate; the eight warps' partials are summed in fixed
+// order, then warp m picks the tile's top-k of row m.
+// ---------------------------------------------------------------------------
+struct VocabArgs {
+  const uint16_t* zt;  // [K, d, 8]
+  float* cand_val;     // [M, K, ntiles, kmax]
+  int* cand_id;
+  float* logits_dbg;   // [M, K, V] or null
+  int d, V, K, kmax, ntiles, units, nstages;
+  int kph[MD_MAX_K];
+};
+
+template <int M>
+__global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
+    heads_vocab_kernel(const __grid_constant__ CUtensorMap wv_map, VocabArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int ns = a.nstages;
+  uint8_t* stage_w = smem;                                              // ns x 32 KB
+  uint8_t* stage_z = smem + size_t(ns) * kStageWBytes;                  // ns x 1 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_z + size_t(ns) * kStageZBytes);
+  uint64_t* empty = full + ns;
+  float* red = reinterpret_cast<float*>(empty + ns);                    // [8][M][256]
+  float* lg = red + kConsumerWarps * M * kTileV;                        // [M][256]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int stages_per_unit = a.d / kStageRows;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ns; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      prefetch_tensormap(&wv_map);
+      const uint64_t pol = policy_evict_first();
+      bool waited_primary = false;
+      int it = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < a.units && ok; unit += gridDim.x) {
+        const int k = unit / a.ntiles, tile = unit % a.ntiles;
+        for (int s = 0; s < stages_per_unit; ++s, ++it) {
+          const int slot = it % ns;
+          if (it >= ns && !mbar_wait(smem_u32(&empty[slot]), ((it / ns) - 1) & 1)) {
+            set_status(MD_DEV_TIMEOUT);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[slot]);
+          mbar_arrive_expect_tx(fb, kStageWBytes + kStageZBytes);
+          tma_load_2d_hint(smem_u32(stage_w + size_t(slot) * kStageWBytes), &wv_map, tile * kTileV,
+                           k * a.d + s * kStageRows, fb, pol);
+          if (!waited_primary) {  // z comes from phase 1: wait for it only now
+            pdl_wait_primary();
+            waited_primary = true;
+          }
+          bulk_load(smem_u32(stage_z + size_t(slot) * kStageZBytes),
+                    a.zt + (size_t(k) * a.d + size_t(s) * kStageRows) * kZPad, kStageZBytes, fb);
+        }
+      }
+      // Drain: wait until the consumers have released every issued stage so
+      // no copy is in flight into shared memory when the CTA exits.
+      for (int j = (it > ns ? it - ns : 0); j < it; ++j) {
+        if (!mbar_wait(smem_u32(&empty[j % ns]), (j / ns) & 1)) {
+          set_status(MD_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------- consumers --------------------------------
+  int it = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x; unit < a.units; unit += gridDim.x) {
+    const int k = unit / a.ntiles, tile = unit % a.ntiles;
+    float acc[M][8];
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[m][c] = 0.f;
+
+    for (int s = 0; s < stages_per_unit; ++s, ++it) {
+      const int slot = it % ns;
+      if (ok && !mbar_wait(smem_u32(&full[slot]), (it / ns) & 1)) {
+        set_status(MD_DEV_TIMEOUT);
+        ok = false;
+      }
+      if (ok) {
+        const uint8_t* wb = stage_w + size_t(slot) * kStageWBytes + warp * 8 * (kTileV * 2) + lane * 16;
+        const uint8_t* zb = stage_z + size_t(slot) * kStageZBytes + warp * 8 * 16;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const uint4 w = *reinterpret_cast<const uint4*>(wb + r * (kTileV * 2));
+          const uint4 zv = *reinterpret_cast<const uint4*>(zb + r * 16);
+          const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            const float zm = (m & 1) ? bf16hi(zw[m >> 1]) : bf16lo(zw[m >> 1]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              acc[m][2 * c] = fmaf(zm, bf16lo(ww[c]), acc[m][2 * c]);
+              acc[m][2 * c + 1] = fmaf(zm, bf16hi(ww[c]), acc[m][2 * c + 1]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
+    }
+
+    // Cross-warp reduction in fixed warp order.
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float4* dst = reinterpret_cast<float4*>(red + (size_t(warp) * M + m) * kTileV + lane * 8);
+      dst[0] = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+      dst[1] = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+    {
+      const int t = threadIdx.x;  // 0..255: one column each
+      const int col = tile * kTileV + t;
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) v += red[(size_t(w) * M + m) * kTileV + t];
+        if (col < a.V) {
+          lg[m * kTileV + t] = v;
+          if (a.logits_dbg) a.logits_dbg[(size_t(m) * a.K + k) * a.V + col] = v;
+        } else {
+          lg[m * kTileV + t] = -INFINITY;
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+
+    // Per-tile top-k of row m by warp m: k rounds, each taking the best entry
+    // strictly after the previous winner in (value desc, id asc) order.
+    if (warp < M) {
+      const int m = warp;
+      float v[kTileV / 32];
+      int id[kTileV / 32];
+#pragma unroll
+      for (int i = 0; i < kTileV / 32; ++i) {
+        const int c = lane + 32 * i;
+        v[i] = lg[m * kTileV + c];
+        id[i] = (tile * kTileV + c < a.V) ? tile * kTileV + c : INT_MAX;
+      }
+      float pv = INFINITY;
+      int pid = -1;
+      const int kk = a.kph[k];
+      const size_t cbase = ((size_t(m) * a.K + k) * a.ntiles + tile) * a.kmax;
+      for (int r = 0; r < kk; ++r) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+#pragma unroll
+        for (int i = 0; i < kTileV / 32; ++i) {
+          if (better(pv, pid, v[i], id[i]) && better(v[i], id[i], bv, bi)) {
+            bv = v[i];
+            bi = id[i];
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (better(ov, oi, bv, bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if (lane == 0) {
+          a.cand_val[cbase + r] = bv;
+          a.cand_id[cbase + r] = (bi == INT_MAX) ? -1 : bi;
+        }
+        pv = bv;
+        pid = bi;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Phase 3: merge the tiles' candidates into each head's top-k.
+// grid (M * K), 256 threads; k rounds of a block-wide "best entry strictly
+// after the previous winner" reduction.
+// ---------------------------------------------------------------------------
+struct MergeArgs {
+  const float* cand_val;
+  const int* cand_id;
+  int32_t* topk_ids;   // [M, K, kmax]
+  float* topk_vals;
+  int K, kmax, ntiles;
+  int kph[MD_MAX_K];
+};
+
+__global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
+  __shared__ float sv[8];
+  __shared__ int si[8];
+  __shared__ float wv;
+  __shared__ int wi;
+  const int mk = blockIdx.x;
+  const int k = mk % a.K;
+  const int kk = a.kph[k];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t base = size_t(mk) * a.ntiles * a.kmax;
+  const int n = a.ntiles * kk;
+  float pv = INFINITY;
+  int pid = -1;
+  for (int r = 0; r < kk; ++r) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    for (int idx = threadIdx.x; idx < n; idx += 256) {
+      const int tile = idx / kk, j = idx - tile * kk;
+      const float cv = a.cand_val[base + size_t(tile) * a.kmax + j];
+      int ci = a.cand_id[base + size_t(tile) * a.kmax + j];
+      if (ci < 0) ci = INT_MAX;
+      if (better(pv, pid, cv, ci) && better(cv, ci, bv, bi)) {
+        bv = cv;
+        bi = ci;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      sv[warp] = bv;
+      si[warp] = bi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      bv = lane < 8 ? sv[lane] : -INFINITY;
+      bi = lane < 8 ? si[lane] : INT_MAX;
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (lane == 0) {
+        wv = bv;
+        wi = bi;
+        a.topk_vals[size_t(mk) * a.kmax + r] = bv;
+        a.topk_ids[size_t(mk) * a.kmax + r] = (bi == INT_MAX) ? -1 : bi;
+      }
+    }
+    __syncthreads();
+    pv = wv;
+    pid = wi;
+  }
+  for (int r = kk + threadIdx.x; r < a.kmax; r += 256) {
+    a.topk_vals[size_t(mk) * a.kmax + r] = -INFINITY;
+    a.topk_ids[size_t(mk) * a.kmax + r] = -1;
+  }
+}
+
+}  // namespace heads
+}  // namespace md

@@ -1,0 +1,420 @@
+// libmedusa: C ABI entry points (validation, launch planning, launches).
+//
+// One translation unit holds every kernel so that the device status word is a
+// single module-scope variable without relocatable device code.
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+#include "heads.cuh"
+#include "tree_build.cuh"
+#include "attention.cuh"
+#include "accept.cuh"
+
+struct md_tree {
+  md::TreeParams tp;
+  int32_t K;
+  int32_t kph[MD_MAX_K];
+};
+
+namespace {
+
+using md::TreeParams;
+
+constexpr int kMaxDevices = 64;
+
+int num_sms() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+md_status cuda_ok(cudaError_t e) {
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MD_ERR_CUDA;
+  }
+  return MD_OK;
+}
+
+md_status last_launch() { return cuda_ok(cudaGetLastError()); }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix; box [box_rows, box_cols].
+md_status make_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                      uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MD_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MD_OK : MD_ERR_CUDA;
+}
+
+template <typename Kernel>
+md_status set_smem(Kernel k, int bytes) {
+  return cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+}
+
+// ----------------------------- heads launchers -----------------------------
+
+template <int M>
+md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
+                       const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
+                       uint8_t* ws, cudaStream_t st) {
+  using namespace md::heads;
+  md_status s;
+  // phase 1
+  W1Args wa;
+  wa.h = h; wa.W1 = W1; wa.b1 = b1;
+  wa.zt = reinterpret_cast<uint16_t*>(ws + pl.off_zt);
+  wa.part = reinterpret_cast<float*>(ws + pl.off_part);
+  wa.counters = reinterpret_cast<int*>(ws + pl.off_cnt);
+  wa.d = pl.d; wa.K = pl.K; wa.splits = pl.splits; wa.rows = pl.rows; wa.ntile_o = pl.ntile_o;
+  if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, size_t(pl.K) * pl.ntile_o * 4, st))) != MD_OK) return s;
+  const int w1_smem = pl.rows * 16 + kConsumerWarps * M * kW1TileO * 4;
+  if ((s = set_smem(heads_w1_kernel<M>, w1_smem)) != MD_OK) return s;
+  heads_w1_kernel<M><<<dim3(pl.ntile_o, pl.splits, pl.K), kW1Threads, w1_smem, st>>>(wa);
+  if ((s = last_launch()) != MD_OK) return s;
+
+  // phase 2 (programmatic dependent launch: its TMA of Wv may start before phase 1 ends)
+  CUtensorMap map;
+  if ((s = make_map_2d(&map, Wv, uint64_t(pl.V), uint64_t(pl.K) * pl.d, kTileV, kStageRows)) != MD_OK) return s;
+  VocabArgs va;
+  va.zt = wa.zt;
+  va.cand_val = reinterpret_cast<float*>(ws + pl.off_cval);
+  va.cand_id = reinterpret_cast<int*>(ws + pl.off_cid);
+  va.logits_dbg = logits_dbg;
+  va.d = pl.d; va.V = pl.V; va.K = pl.K; va.kmax = pl.kmax; va.ntiles = pl.ntiles; va.units = pl.units;
+  va.nstages = pl.nstages;
+  for (int k = 0; k < MD_MAX_K; ++k) va.kph[k] = k < pl.K ? kph[k] : 0;
+  const int v_smem = vocab_smem_bytes(M, pl.nstages);
+  if ((s = set_smem(heads_vocab_kernel<M>, v_smem)) != MD_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(num_sms(), pl.units));
+  cfg.blockDim = dim3((kConsumerWarps + 1) * 32);
+  cfg.dynamicSmemBytes = v_smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if ((s = cuda_ok(cudaLaunchKernelEx(&cfg, heads_vocab_kernel<M>, map, va))) != MD_OK) return s;
+
+  // phase 3
+  MergeArgs ma;
+  ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
+  ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
+  ma.K = pl.K; ma.kmax = pl.kmax; ma.ntiles = pl.ntiles;
+  for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
+  heads_merge_kernel<<<pl.M * pl.K, 256, 0, st>>>(ma);
+  return last_launch();
+}
+
+md_status heads_check(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax) {
+  if (M <= 0 || d <= 0 || V <= 0 || K <= 0 || kmax <= 0) return MD_ERR_INVALID_ARG;
+  if (K > MD_MAX_K || kmax > MD_MAX_KMAX) return MD_ERR_UNSUPPORTED;
+  if (M > md::heads::kMaxM) return MD_ERR_UNSUPPORTED;
+  if (d % 64 != 0 || V % 8 != 0 || V < 256) return MD_ERR_UNSUPPORTED;
+  if (size_t(K) * d >= (size_t(1) << 31) || V >= (1 << 30)) return MD_ERR_UNSUPPORTED;
+  return MD_OK;
+}
+
+// ---------------------------- accept planning ------------------------------
+
+struct AcceptPlan {
+  int nchunks, chunk_len;
+  size_t bytes;
+};
+
+AcceptPlan accept_plan(int B, int T, int V) {
+  AcceptPlan p;
+  const int rows = B * T;
+  const int max_chunks = (V + 1023) / 1024;
+  int n = (2 * num_sms() + rows - 1) / rows;
+  n = std::max(1, std::min(n, max_chunks));
+  int len = (V + n - 1) / n;
+  len = (len + 1023) / 1024 * 1024;
+  p.chunk_len = len;
+  p.nchunks = (V + len - 1) / len;
+  p.bytes = size_t(rows) * p.nchunks * md::acc::kPartFloats * 4;
+  return p;
+}
+
+// --------------------------- attention planning ----------------------------
+
+struct AttnPlan {
+  int G, R, max_chunks;
+  size_t off_ml, bytes;
+};
+
+AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
+  AttnPlan p;
+  p.G = Hq / Hkv;
+  p.R = T * p.G;
+  p.max_chunks = (S_max + md::attn::kChunk - 1) / md::attn::kChunk;
+  const size_t rows = size_t(B) * Hkv * p.max_chunks * p.R;
+  p.off_ml = md::heads::align256(rows * dh * 4);
+  p.bytes = p.off_ml + md::heads::align256(rows * 8);
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+md_status md_tree_create(const int32_t* parent, const int32_t* head_rank, int32_t T, int32_t K,
+                         const int32_t* k_per_head, md_tree** out) {
+  if (!parent || !head_rank || !k_per_head || !out) return MD_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (T < 1 || T > MD_MAX_T || K < 1 || K > MD_MAX_K) return MD_ERR_INVALID_ARG;
+  if (parent[0] != -1) return MD_ERR_INVALID_ARG;
+  for (int k = 0; k < K; ++k)
+    if (k_per_head[k] < 1 || k_per_head[k] > MD_MAX_KMAX) return MD_ERR_INVALID_ARG;
+  md_tree* t = new (std::nothrow) md_tree;
+  if (!t) return MD_ERR_INVALID_ARG;
+  std::memset(t, 0, sizeof(*t));
+  TreeParams& tp = t->tp;
+  tp.T = T;
+  tp.W = (T + 31) / 32;
+  tp.K = K;
+  t->K = K;
+  for (int k = 0; k < K; ++k) t->kph[k] = k_per_head[k];
+  tp.parent[0] = -1;
+  tp.depth[0] = 0;
+  tp.rank[0] = 0;
+  tp.anc[0][0] = 1u;
+  int maxd = 0;
+  for (int j = 1; j < T; ++j) {
+    const int p = parent[j];
+    if (p < 0 || p >= j) { delete t; return MD_ERR_INVALID_ARG; }
+    const int d = tp.depth[p] + 1;
+    if (d > K) { delete t; return MD_ERR_INVALID_ARG; }
+    const int r = head_rank[j];
+    if (r < 0 || r >= k_per_head[d - 1]) { delete t; return MD_ERR_INVALID_ARG; }
+    for (int i = 1; i < j; ++i)
+      if (parent[i] == p && head_rank[i] == r) { delete t; return MD_ERR_INVALID_ARG; }
+    tp.parent[j] = int8_t(p);
+    tp.depth[j] = int8_t(d);
+    tp.rank[j] = int8_t(r);
+    for (int w = 0; w < 4; ++w) tp.anc[j][w] = tp.anc[p][w];
+    tp.anc[j][j >> 5] |= 1u << (j & 31);
+    maxd = d > maxd ? d : maxd;
+  }
+  tp.max_depth = maxd;
+  *out = t;
+  return MD_OK;
+}
+
+md_status md_tree_destroy(md_tree* tree) {
+  delete tree;
+  return MD_OK;
+}
+
+md_status md_tree_info(const md_tree* tree, int32_t* T, int32_t* max_depth) {
+  if (!tree) return MD_ERR_INVALID_ARG;
+  if (T) *T = tree->tp.T;
+  if (max_depth) *max_depth = tree->tp.max_depth;
+  return MD_OK;
+}
+
+md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax, size_t* bytes) {
+  if (!bytes) return MD_ERR_INVALID_ARG;
+  md_status s = heads_check(M, d, V, K, kmax);
+  if (s != MD_OK) return s;
+  *bytes = md::heads::make_plan(M, d, V, K, kmax, num_sms()).bytes;
+  return MD_OK;
+}
+
+md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, int32_t M,
+                          int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax,
+                          int32_t* topk_ids, float* topk_vals, float* logits_dbg, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
+  md_status s = heads_check(M, d, V, K, kmax);
+  if (s != MD_OK) return s;
+  for (int k = 0; k < K; ++k)
+    if (k_per_head[k] < 1 || k_per_head[k] > kmax || k_per_head[k] > V) return MD_ERR_INVALID_ARG;
+  if (!aligned(h, 2) || !aligned(W1, 16) || !aligned(b1, 2) || !aligned(Wv, 16) || !aligned(topk_ids, 4) ||
+      !aligned(topk_vals, 4) || (logits_dbg && !aligned(logits_dbg, 4)))
+    return MD_ERR_INVALID_ARG;
+  const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
+  if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  switch (M) {
+    case 1: return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 2: return launch_heads<2>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 3: return launch_heads<3>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 4: return launch_heads<4>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 5: return launch_heads<5>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 6: return launch_heads<6>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 7: return launch_heads<7>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    case 8: return launch_heads<8>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    default: return MD_ERR_UNSUPPORTED;
+  }
+}
+
+md_status md_tree_build(const md_tree* tree, const int32_t* topk_ids, int32_t M, int32_t kmax,
+                        const int32_t* head_row, const int32_t* root_token, const int32_t* prefix_len, int32_t B,
+                        int32_t* tokens, int32_t* parent, uint32_t* anc, int32_t* pos, void* stream) {
+  if (!tree || !topk_ids || !root_token || !prefix_len || !tokens || !parent || !anc || !pos)
+    return MD_ERR_INVALID_ARG;
+  if (M < 1 || B < 1 || kmax < 1 || kmax > MD_MAX_KMAX) return MD_ERR_INVALID_ARG;
+  if (!head_row && M < B) return MD_ERR_INVALID_ARG;
+  for (int k = 0; k < tree->K; ++k)
+    if (tree->kph[k] > kmax) return MD_ERR_INVALID_ARG;
+  md::tree::BuildArgs a;
+  a.topk_ids = topk_ids; a.head_row = head_row; a.root_token = root_token; a.prefix_len = prefix_len;
+  a.tokens = tokens; a.parent = parent; a.anc = anc; a.pos = pos;
+  a.M = M; a.K = tree->K; a.kmax = kmax;
+  md::tree::tree_build_kernel<<<B, MD_MAX_T, 0, static_cast<cudaStream_t>(stream)>>>(tree->tp, a);
+  return last_launch();
+}
+
+md_status md_attention_workspace(int32_t B, int32_t T, int32_t Hq, int32_t Hkv, int32_t dh, int32_t S_max,
+                                 size_t* bytes) {
+  if (!bytes || B < 1 || T < 1 || Hq < 1 || Hkv < 1 || S_max < 1) return MD_ERR_INVALID_ARG;
+  if (T > MD_MAX_T || (dh != 64 && dh != 128) || Hq % Hkv != 0 || Hq / Hkv > 16) return MD_ERR_UNSUPPORTED;
+  *bytes = attn_plan(B, T, Hq, Hkv, dh, S_max).bytes;
+  return MD_OK;
+}
+
+md_status md_tree_attention(const md_bf16* q, const md_bf16* k_cache, const md_bf16* v_cache,
+                            const int32_t* prefix_len, int32_t S_max, const md_tree* tree, int32_t B, int32_t Hq,
+                            int32_t Hkv, int32_t dh, float scale, float* out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  if (!q || !k_cache || !v_cache || !prefix_len || !tree || !out) return MD_ERR_INVALID_ARG;
+  const int T = tree->tp.T;
+  size_t need = 0;
+  md_status s = md_attention_workspace(B, T, Hq, Hkv, dh, S_max, &need);
+  if (s != MD_OK) return s;
+  if (S_max < T || !(scale >= 0.f) || !std::isfinite(scale)) return MD_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+    return MD_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  const AttnPlan pl = attn_plan(B, T, Hq, Hkv, dh, S_max);
+  md::attn::Args a;
+  a.q = q; a.kc = k_cache; a.vc = v_cache; a.prefix_len = prefix_len;
+  a.part_acc = static_cast<float*>(ws);
+  a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
+  a.out = out;
+  a.S_max = S_max; a.Hq = Hq; a.Hkv = Hkv; a.G = pl.G; a.R = pl.R; a.max_chunks = pl.max_chunks;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(float(dh));
+  a.scale_log2 = sc * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(pl.max_chunks, Hkv, B);
+  if (dh == 128) {
+    constexpr int sm = md::attn::smem_bytes<128>();
+    if ((s = set_smem(md::attn::attn_chunk_kernel<128>, sm)) != MD_OK) return s;
+    md::attn::attn_chunk_kernel<128><<<grid, md::attn::kThreads, sm, st>>>(tree->tp, a);
+    if ((s = last_launch()) != MD_OK) return s;
+    md::attn::attn_merge_kernel<128><<<dim3(T * Hq, B), 128, 0, st>>>(tree->tp, a);
+  } else {
+    constexpr int sm = md::attn::smem_bytes<64>();
+    if ((s = set_smem(md::attn::attn_chunk_kernel<64>, sm)) != MD_OK) return s;
+    md::attn::attn_chunk_kernel<64><<<grid, md::attn::kThreads, sm, st>>>(tree->tp, a);
+    if ((s = last_launch()) != MD_OK) return s;
+    md::attn::attn_merge_kernel<64><<<dim3(T * Hq, B), 64, 0, st>>>(tree->tp, a);
+  }
+  return last_launch();
+}
+
+md_status md_accept_workspace(int32_t B, int32_t T, int32_t V, size_t* bytes) {
+  if (!bytes || B < 1 || T < 1 || V < 1) return MD_ERR_INVALID_ARG;
+  if (T > MD_MAX_T || V % 8 != 0) return MD_ERR_UNSUPPORTED;
+  *bytes = accept_plan(B, T, V).bytes;
+  return MD_OK;
+}
+
+md_status md_tree_accept(const float* logits, int32_t V, const int32_t* tokens, const md_tree* tree, int32_t B,
+                         int32_t K, int32_t mode, float temperature, float eps, float alpha, int32_t* accept_len,
+                         int32_t* path, int32_t* bonus, void* ws, size_t ws_bytes, void* stream) {
+  if (!logits || !tokens || !tree || !accept_len || !path || !bonus) return MD_ERR_INVALID_ARG;
+  const int T = tree->tp.T;
+  size_t need = 0;
+  md_status s = md_accept_workspace(B, T, V, &need);
+  if (s != MD_OK) return s;
+  if (K < tree->tp.max_depth || K < 0) return MD_ERR_INVALID_ARG;
+  if (mode != MD_ACCEPT_GREEDY && mode != MD_ACCEPT_TYPICAL) return MD_ERR_INVALID_ARG;
+  if (mode == MD_ACCEPT_TYPICAL &&
+      (!(temperature > 0.f) || !std::isfinite(temperature) || !(eps >= 0.f) || !(alpha >= 0.f)))
+    return MD_ERR_INVALID_ARG;
+  if (!aligned(logits, 16)) return MD_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  const AcceptPlan pl = accept_plan(B, T, V);
+  md::acc::Args a;
+  a.logits = logits; a.tokens = tokens; a.accept_len = accept_len; a.path = path; a.bonus = bonus;
+  a.part = static_cast<float*>(ws);
+  a.T = T; a.V = V; a.K = K; a.nchunks = pl.nchunks; a.chunk_len = pl.chunk_len; a.mode = mode;
+  a.inv_temp = mode == MD_ACCEPT_TYPICAL ? 1.0f / temperature : 1.0f;
+  a.log_eps = std::log(eps);
+  a.log_alpha = std::log(alpha);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  md::acc::accept_rows_kernel<<<dim3(pl.nchunks, B * T), md::acc::kRowThreads, 0, st>>>(a);
+  if ((s = last_launch()) != MD_OK) return s;
+  md::acc::accept_walk_kernel<<<B, MD_MAX_T, 0, st>>>(tree->tp, a);
+  return last_launch();
+}
+
+md_status md_get_device_status(void* stream, int32_t* out, int32_t clear) {
+  if (!out) return MD_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  md_status s;
+  if ((s = cuda_ok(cudaStreamSynchronize(st))) != MD_OK) return s;
+  int v = 0;
+  if ((s = cuda_ok(cudaMemcpyFromSymbol(&v, md::g_device_status, sizeof(int)))) != MD_OK) return s;
+  *out = v;
+  if (clear) {
+    const int zero = 0;
+    if ((s = cuda_ok(cudaMemcpyToSymbol(md::g_device_status, &zero, sizeof(int)))) != MD_OK) return s;
+  }
+  return MD_OK;
+}
+
+const char* md_status_string(md_status status) {
+  switch (status) {
+    case MD_OK: return "ok";
+    case MD_ERR_INVALID_ARG: return "invalid argument";
+    case MD_ERR_UNSUPPORTED: return "unsupported size or layout";
+    case MD_ERR_CUDA: return "CUDA runtime error";
+    case MD_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MD_ERR_TIMEOUT: return "a bounded device wait gave up";
+    default: return "unknown status";
+  }
+}
+
+int32_t md_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+"""One Medusa draft-and-verify step through the C ABI.
+
+Owns the output buffers and workspaces of the four calls and issues them in
+order on one stream: heads + top-k -> tree build -> tree attention (one layer
+of the verification pass) -> acceptance. No arithmetic happens here.
+"""
+from __future__ import annotations
+
+import torch
+
+from .binding import (Tree, accept_workspace_bytes, attention_workspace_bytes, heads_workspace_bytes,
+                      medusa_heads, tree_accept, tree_attention, tree_build, workspace)
+from .tree_spec import tree_arrays
+
+
+class MedusaStep:
+    def __init__(self, *, B, M, d, V, K, k_per_head, tree_tuples, Hq, Hkv, dh, S_max, mode="greedy",
+                 temperature=0.7, eps=0.09, alpha=0.3, device="cuda", keep_logits=False):
+        parent, rank = tree_arrays(tree_tuples)
+        self.tree = Tree(parent, rank, k_per_head)
+        self.B, self.M, self.d, self.V, self.K = B, M, d, V, K
+        self.k_per_head = list(k_per_head)
+        self.kmax = max(k_per_head)
+        self.T = self.tree.T
+        self.Hq, self.Hkv, self.dh, self.S_max = Hq, Hkv, dh, S_max
+        self.mode, self.temperature, self.eps, self.alpha = mode, temperature, eps, alpha
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.topk_ids = torch.empty((M, K, self.kmax), **i32)
+        self.topk_vals = torch.empty((M, K, self.kmax), **f32)
+        self.logits_dbg = torch.empty((M, K, V), **f32) if keep_logits else None
+        self.tokens = torch.empty((B, self.T), **i32)
+        self.parent = torch.empty((self.T,), **i32)
+        self.anc = torch.empty((self.T, (self.T + 31) // 32), **i32)
+        self.pos = torch.empty((B, self.T), **i32)
+        self.attn_out = torch.empty((B, self.T, Hq, dh), **f32)
+        self.accept_len = torch.empty((B,), **i32)
+        self.path = torch.empty((B, K + 1), **i32)
+        self.bonus = torch.empty((B,), **i32)
+        self.ws_heads = workspace(heads_workspace_bytes(M, d, V, K, self.kmax), dev)
+        self.ws_attn = workspace(attention_workspace_bytes(B, self.T, Hq, Hkv, dh, S_max), dev)
+        self.ws_acc = workspace(accept_workspace_bytes(B, self.T, V), dev)
+
+    def heads(self, h, W1, b1, Wv, stream=None):
+        medusa_heads(h, W1, b1, Wv, self.k_per_head, self.topk_ids, self.topk_vals, self.ws_heads,
+                     logits_dbg=self.logits_dbg, stream=stream)
+
+    def build(self, root_token, prefix_len, head_row=None, stream=None):
+        tree_build(self.tree, self.topk_ids, root_token, prefix_len, self.tokens, self.parent, self.anc,
+                   self.pos, head_row=head_row, stream=stream)
+
+    def attention(self, q, k_cache, v_cache, prefix_len, stream=None):
+        tree_attention(q, k_cache, v_cache, prefix_len, self.tree, self.attn_out, self.ws_attn, stream=stream)
+
+    def accept(self, logits, stream=None):
+        tree_accept(logits, self.tokens, self.tree, self.accept_len, self.path, self.bonus, self.ws_acc,
+                    mode=self.mode, temperature=self.temperature, eps=self.eps, alpha=self.alpha, stream=stream)
+
+    def run(self, h, W1, b1, Wv, root_token, prefix_len, q, k_cache, v_cache, logits, head_row=None,
+            stream=None):
+        self.heads(h, W1, b1, Wv, stream)
+        self.build(root_token, prefix_len, head_row, stream)
+        self.attention(q, k_cache, v_cache, prefix_len, stream)
+        self.accept(logits, stream)

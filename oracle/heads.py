@@ -57,15 +57,29 @@ def silu(u: np.ndarray) -> np.ndarray:
         return u / (1.0 + np.exp(-u))
 
 
-def residual_block(h_bits, W1_bits, b1_bits) -> np.ndarray:
-    """z[m, k, :] = bf16(h[m] + SiLU(h[m] W1[k] + b1[k])) as bf16 bits [M, K, d]."""
+def residual_block(h_bits, W1_bits, b1_bits, cols=None) -> np.ndarray:
+    """z[m, k, :] = bf16(h[m] + SiLU(h[m] W1[k] + b1[k])) as bf16 bits [M, K, d].
+
+    ``cols`` optionally restricts the output to those hidden units (the
+    result is then [M, K, len(cols)]).
+    """
+    d = h_bits.shape[1]
+    cols = np.arange(d) if cols is None else np.asarray(cols)
+    return residual_block_columns(h_bits, W1_bits[:, :, cols], b1_bits[:, cols], cols)
+
+
+def residual_block_columns(h_bits, W1c_bits, b1c_bits, cols) -> np.ndarray:
+    """The residual block for the hidden units ``cols`` only, given their
+    weight columns ``W1c[k] = W1[k][:, cols]`` and biases ``b1c[k] = b1[k][cols]``.
+    Returns z bits [M, K, len(cols)]."""
     h = bf16_to_f64(h_bits)                                   # [M, d]
-    K = W1_bits.shape[0]
-    M, d = h.shape
-    z = np.empty((M, K, d), dtype=np.uint16)
+    K = W1c_bits.shape[0]
+    M = h.shape[0]
+    cols = np.asarray(cols)
+    z = np.empty((M, K, len(cols)), dtype=np.uint16)
     for k in range(K):
-        u = h @ bf16_to_f64(W1_bits[k]) + bf16_to_f64(b1_bits[k])[None, :]
-        z[:, k, :] = f64_to_bf16(h + silu(u))
+        u = h @ bf16_to_f64(W1c_bits[k]) + bf16_to_f64(b1c_bits[k])[None, :]
+        z[:, k, :] = f64_to_bf16(h[:, cols] + silu(u))
     return z
 
 

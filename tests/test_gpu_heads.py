@@ -1,0 +1,93 @@
+"""GPU parity of md_medusa_heads against the oracle (B200 only)."""
+import numpy as np
+import pytest
+
+from oracle import heads as oh
+from seeded_inputs import gen
+
+from .helpers import HEADS_RTOL, bf16_tensor, check_topk_row, head_weights, normwise
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _run(h, W1, b1, Wv, kph, kmax=None, dbg=True):
+    import medusa_draft_heads_b200 as md
+    M, d = h.shape
+    K, _, V = Wv.shape
+    kmax = kmax or max(kph)
+    ids = torch.full((M, K, kmax), -7, dtype=torch.int32, device="cuda")
+    vals = torch.zeros((M, K, kmax), dtype=torch.float32, device="cuda")
+    logits = torch.zeros((M, K, V), dtype=torch.float32, device="cuda") if dbg else None
+    ws = md.workspace(md.heads_workspace_bytes(M, d, V, K, kmax))
+    md.medusa_heads(bf16_tensor(h), bf16_tensor(W1), bf16_tensor(b1), bf16_tensor(Wv), kph, ids, vals, ws,
+                    logits_dbg=logits)
+    torch.cuda.synchronize()
+    assert md.device_status() == 0
+    return ids.cpu().numpy(), vals.cpu().numpy(), (logits.cpu().numpy() if dbg else None)
+
+
+@pytest.mark.parametrize("M,d,V,kph", [(1, 256, 1024, (4, 3, 2, 2)), (2, 512, 1000, (10, 10, 10, 10)),
+                                       (8, 320, 2056, (16, 1, 7, 3)), (3, 1024, 4096, (5, 5, 5, 5))])
+def test_heads_match_oracle_small(M, d, V, kph):
+    h, W1, b1, Wv = head_weights(11 + M, d, V, len(kph), M)
+    ids, vals, logits = _run(h, W1, b1, Wv, kph, kmax=max(kph) + 1)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph, max(kph) + 1)
+    err = normwise(logits, rlog)
+    assert err.max() <= HEADS_RTOL, err.max()
+    assert err.max() <= 1e-4        # fp32 accumulation is far inside the stated bound
+    for m in range(M):
+        for k, kk in enumerate(kph):
+            check_topk_row(ids[m, k], vals[m, k], rlog[m, k], kk)
+            assert np.all(ids[m, k, kk:] == -1) and np.all(np.isneginf(vals[m, k, kk:]))
+
+
+def _integer_heads(seed, M, d, V, K):
+    """h, Wv small integers and W1 = b1 = 0: z = h exactly and every logit is
+    an integer both sides compute exactly, with many exact ties."""
+    rng = np.random.default_rng(seed)
+    hv = rng.integers(-2, 3, (M, d)).astype(np.float32)
+    wv = rng.integers(-1, 2, (K, d, V)).astype(np.float32)
+    h = gen.f32_to_bf16_bits(hv)
+    Wv = gen.f32_to_bf16_bits(wv)
+    W1 = np.zeros((K, d, d), dtype=np.uint16)
+    b1 = np.zeros((K, d), dtype=np.uint16)
+    return h, W1, b1, Wv
+
+
+@pytest.mark.parametrize("M,d,V,kph", [(1, 128, 1024, (16, 10, 1, 5)), (4, 256, 1000, (3, 16, 2, 9)),
+                                       (8, 64, 776, (16, 16, 16, 16))])
+def test_topk_bit_exact_on_exact_integer_logits(M, d, V, kph):
+    h, W1, b1, Wv = _integer_heads(M * 7 + d, M, d, V, len(kph))
+    ids, vals, logits = _run(h, W1, b1, Wv, kph)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph)
+    assert np.array_equal(logits, rlog.astype(np.float32))
+    assert np.array_equal(ids, rid)
+    assert np.array_equal(vals, rval.astype(np.float32))
+    # ties really were exercised
+    ties = sum(int(np.sum(rlog[m, k] == rval[m, k, kk - 1])) > 1
+               for m in range(M) for k, kk in enumerate(kph))
+    assert ties > 0
+
+
+def test_heads_are_deterministic():
+    h, W1, b1, Wv = head_weights(5, 512, 2048, 4, 2)
+    a = _run(h, W1, b1, Wv, (10, 10, 10, 10))
+    b = _run(h, W1, b1, Wv, (10, 10, 10, 10))
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_heads_reject_bad_arguments():
+    import medusa_draft_heads_b200 as md
+    h, W1, b1, Wv = head_weights(1, 256, 1024, 4, 1)
+    ids = torch.zeros((1, 4, 4), dtype=torch.int32, device="cuda")
+    vals = torch.zeros((1, 4, 4), dtype=torch.float32, device="cuda")
+    ws = md.workspace(64)
+    with pytest.raises(md.MedusaError, match="workspace"):
+        md.medusa_heads(bf16_tensor(h), bf16_tensor(W1), bf16_tensor(b1), bf16_tensor(Wv), (4, 3, 2, 2), ids,
+                        vals, ws)
+    ws = md.workspace(md.heads_workspace_bytes(1, 256, 1024, 4, 4))
+    with pytest.raises(md.MedusaError, match="invalid"):
+        md.medusa_heads(bf16_tensor(h), bf16_tensor(W1), bf16_tensor(b1), bf16_tensor(Wv), (5, 3, 2, 2), ids,
+                        vals, ws)

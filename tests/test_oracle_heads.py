@@ -179,3 +179,12 @@ def test_zero_block_reduces_to_plain_projection(w_scale):
         assert np.max(np.abs(logits[0, k] - exact)) <= 1e-14
         brute = sorted(range(V), key=lambda v: (-exact[v], v))[:5]
         assert list(ids[0, k]) == brute
+
+
+def test_residual_block_column_subset_agrees():
+    d, K = 128, 2
+    h, W1, b1, _ = (gen.normal_bf16(2, "h", (2, d), 1.0), gen.normal_bf16(2, "W1", (K, d, d), 0.02),
+                    gen.normal_bf16(2, "b1", (K, d), 0.02), None)
+    full = oh.residual_block(h, W1, b1)
+    cols = [5, 0, 127, 64]
+    assert np.array_equal(oh.residual_block(h, W1, b1, cols=cols), full[:, :, cols])
