@@ -71,7 +71,8 @@ enum {
 
 /* Supported ranges (anything else: MD_ERR_UNSUPPORTED).
  *   heads:     1 <= K <= 8, 1 <= k_i <= kmax <= 16, d % 64 == 0, V % 8 == 0,
- *              V >= 256, 1 <= M <= 8 on the streaming path.
+ *              V >= 256, 1 <= M <= 4096 (M <= 8: CUDA-core weight stream;
+ *              M > 8: tcgen05 tensor-core GEMM, h and b1 16-byte aligned).
  *   tree:      1 <= T <= 128, depth <= K.
  *   attention: dh in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16.
  */

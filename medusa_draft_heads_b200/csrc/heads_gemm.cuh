@@ -1,0 +1,275 @@
+// Medusa draft heads on the tensor cores (tcgen05), for many hidden rows.
+//
+// Source: "Medusa heads versus separate draft model", sections "What each one
+// is" and "Cost per step" (the same head computation as heads.cuh). Once the
+// heads run on many rows at once -- every tree node of a batch of requests,
+// e.g. 8 x 65 = 520 rows -- the projection stops being a weight stream and
+// becomes a dense GEMM (the page's tree paragraph: past the ridge point the
+// verification width turns the step compute-bound). Both phases then run as
+// one persistent tcgen05 GEMM each:
+//
+//   phase 1  D = h   . W1_k   (M x d x d)   epilogue: z = bf16(h + SiLU(D + b1))
+//   phase 2  D = z_k . Wv_k   (M x d x V)   epilogue: per-row top-k of the tile
+//
+// CTA tile 128 x 256 (UMMA M = 128, N = 256, K = 16 per instruction), 64-deep
+// K stages of A (16 KB, K-major) and B (4 x 8 KB, N-major, straight from the
+// input-major weights) brought in by TMA with 128-byte swizzle. Warp 0 feeds
+// TMA, one thread of warp 1 issues tcgen05.mma into one of two 128 x 256 fp32
+// accumulators in tensor memory (512 columns), warps 2..5 drain the other
+// accumulator through tcgen05.ld (one TMEM lane = one row per thread).
+#pragma once
+
+#include "common.cuh"
+
+namespace md {
+namespace gemm {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = kBM * kBK * 2;     // 16 KB
+constexpr uint32_t kBBox = kBK * 64 * 2;        // 8 KB: 64 k-rows x 64 n-columns
+constexpr uint32_t kBBytes = 4 * kBBox;         // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxM = 4096;
+
+enum { EPI_SILU = 0, EPI_TOPK = 1 };
+
+struct Args {
+  int M, d, N, K;                 // rows, reduction length, output columns, heads
+  int mtiles, ntiles, tiles;
+  int a_shared;                   // A is one matrix for every head (phase 1: h)
+  const uint16_t* h;              // [M, d]      phase 1 residual
+  const uint16_t* b1;             // [K, d]      phase 1 bias
+  uint16_t* zg;                   // [K, M, d]   phase 1 output
+  float* cand_val;                // [M, K, ntiles, kmax]  phase 2 output
+  int* cand_id;
+  float* logits_dbg;              // [M, K, N] or null
+  int kmax;
+  int kph[MD_MAX_K];
+};
+
+template <int KK>
+struct TopK {
+  float v[KK];
+  int i[KK];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < KK; ++j) {
+      v[j] = -INFINITY;
+      i[j] = INT_MAX;
+    }
+  }
+  __device__ __forceinline__ void push(float x, int id) {
+    if (!better(x, id, v[KK - 1], i[KK - 1])) return;
+    v[KK - 1] = x;
+    i[KK - 1] = id;
+#pragma unroll
+    for (int j = KK - 1; j > 0; --j) {
+      if (better(v[j], i[j], v[j - 1], i[j - 1])) {
+        const float tv = v[j];
+        v[j] = v[j - 1];
+        v[j - 1] = tv;
+        const int ti = i[j];
+        i[j] = i[j - 1];
+        i[j - 1] = ti;
+      }
+    }
+  }
+};
+
+template <int EPI, int KK>
+__global__ void __launch_bounds__(kThreads, 1)
+    heads_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = a.d / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 4);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------- TMA producer -------------------------------
+    if (lane == 0) {
+      prefetch_tensormap(&amap);
+      prefetch_tensormap(&bmap);
+      pdl_wait_primary();   // A may be the previous kernel's output
+      const uint64_t pol = policy_evict_first();
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+        const int mt = tile % a.mtiles, r = tile / a.mtiles;
+        const int nt = r % a.ntiles, k = r / a.ntiles;
+        for (int s = 0; s < nk; ++s, ++it) {
+          const int slot = it % kStages;
+          if (it >= kStages && !mbar_wait(smem_u32(&empty[slot]), ((it / kStages) - 1) & 1)) {
+            set_status(MD_DEV_TIMEOUT);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[slot]);
+          uint8_t* st = smem + size_t(slot) * kStageBytes;
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_3d(smem_u32(st), &amap, s * kBK, mt * kBM, a.a_shared ? 0 : k, fb);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tma_load_3d_hint(smem_u32(st + kABytes + j * kBBox), &bmap, nt * kBN + j * 64, s * kBK, k, fb, pol);
+        }
+      }
+      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j) {
+        if (!mbar_wait(smem_u32(&empty[j % kStages]), (j / kStages) & 1)) {
+          set_status(MD_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------- MMA issuer ---------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, kBN, 0, 1);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        if (lt >= 2 && !mbar_wait(smem_u32(&acc_empty[buf]), ((lt >> 1) - 1) & 1)) {
+          set_status(MD_DEV_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + uint32_t(buf * kBN);
+        for (int s = 0; s < nk; ++s, ++it) {
+          const int slot = it % kStages;
+          if (!mbar_wait(smem_u32(&full[slot]), (it / kStages) & 1)) {
+            set_status(MD_DEV_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + size_t(slot) * kStageBytes);
+          const uint64_t adesc = umma_desc_sw128(sa, 16, 1024);
+          const uint64_t bdesc = umma_desc_sw128(sa + kABytes, kBBox, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_f16(d_tmem, adesc + uint64_t((kk * 32) >> 4), bdesc + uint64_t((kk * 2048) >> 4), idesc,
+                     (s | kk) != 0);
+          umma_commit(smem_u32(&empty[slot]));
+        }
+        umma_commit(smem_u32(&acc_full[buf]));
+      }
+    }
+  } else {
+    // -------------------------------- epilogue ----------------------------------
+    const int q = warp & 3;   // TMEM lanes 32q .. 32q+31 belong to this warp
+    const int row = q * 32 + lane;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++lt) {
+      const int mt = tile % a.mtiles, r = tile / a.mtiles;
+      const int nt = r % a.ntiles, k = r / a.ntiles;
+      const int buf = lt & 1;
+      if (!mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1)) {
+        set_status(MD_DEV_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int m = mt * kBM + row;
+      const bool live = m < a.M;
+      const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * kBN);
+      if constexpr (EPI == EPI_SILU) {
+        for (int c = 0; c < kBN; c += 32) {
+          float v[32];
+          tmem_ld32(tbase + c, v);
+          const int o0 = nt * kBN + c;
+          if (live && o0 < a.d) {
+            const uint4* hp = reinterpret_cast<const uint4*>(a.h + size_t(m) * a.d + o0);
+            const uint4* bp = reinterpret_cast<const uint4*>(a.b1 + size_t(k) * a.d + o0);
+            uint4* zp = reinterpret_cast<uint4*>(a.zg + (size_t(k) * a.M + m) * a.d + o0);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint4 hv = hp[g], bv = __ldg(bp + g);
+              const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+              const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+              uint32_t zw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float u0 = v[g * 8 + 2 * e] + bf16lo(bw[e]);
+                const float u1 = v[g * 8 + 2 * e + 1] + bf16hi(bw[e]);
+                const uint16_t z0 = f32_to_bf16_rne(bf16lo(hw[e]) + u0 / (1.0f + expf(-u0)));
+                const uint16_t z1 = f32_to_bf16_rne(bf16hi(hw[e]) + u1 / (1.0f + expf(-u1)));
+                zw[e] = uint32_t(z0) | (uint32_t(z1) << 16);
+              }
+              zp[g] = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+            }
+          }
+        }
+      } else {
+        TopK<KK> tk;
+        tk.init();
+        for (int c = 0; c < kBN; c += 32) {
+          float v[32];
+          tmem_ld32(tbase + c, v);
+          const int c0 = nt * kBN + c;
+          if (live) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < a.N) tk.push(v[j], c0 + j);
+            if (a.logits_dbg) {
+              float* lp = a.logits_dbg + (size_t(m) * a.K + k) * a.N + c0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                if (c0 + j < a.N) *reinterpret_cast<float4*>(lp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+          }
+        }
+        if (live) {
+          const int kk = a.kph[k];
+          const size_t cb = ((size_t(m) * a.K + k) * a.ntiles + nt) * a.kmax;
+#pragma unroll
+          for (int j = 0; j < KK; ++j) {
+            if (j < kk) {
+              a.cand_val[cb + j] = tk.v[j];
+              a.cand_id[cb + j] = tk.i[j] == INT_MAX ? -1 : tk.i[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace gemm
+}  // namespace md

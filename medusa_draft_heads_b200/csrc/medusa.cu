@@ -8,8 +8,10 @@
 
 #include "common.cuh"
 #include "heads.cuh"
+#include "heads_gemm.cuh"
 #include "tree_build.cuh"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "accept.cuh"
 
 struct md_tree {
@@ -142,10 +144,104 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   return last_launch();
 }
 
+// Workspace of the tensor-core path (M > 8): z [K, M, d] bf16 and the
+// per-tile candidates [M, K, ceil(V/256), kmax].
+struct GemmPlan {
+  int mtiles, ntiles1, ntiles2;
+  size_t off_z, off_cval, off_cid, bytes;
+};
+
+GemmPlan gemm_plan(int M, int d, int V, int K, int kmax) {
+  using md::heads::align256;
+  GemmPlan p;
+  p.mtiles = (M + md::gemm::kBM - 1) / md::gemm::kBM;
+  p.ntiles1 = (d + md::gemm::kBN - 1) / md::gemm::kBN;
+  p.ntiles2 = (V + md::gemm::kBN - 1) / md::gemm::kBN;
+  size_t o = 0;
+  p.off_z = o;    o = align256(o + size_t(K) * M * d * 2);
+  p.off_cval = o; o = align256(o + size_t(M) * K * p.ntiles2 * kmax * 4);
+  p.off_cid = o;  o = align256(o + size_t(M) * K * p.ntiles2 * kmax * 4);
+  p.bytes = o;
+  return p;
+}
+
+// 3-D bf16 tensor map over [n2][n1][n0] (n0 contiguous), box [1][b1][b0], 128-byte swizzle.
+md_status make_map_3d_sw128(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0,
+                            uint32_t b1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MD_ERR_CUDA;
+  cuuint64_t dims[3] = {n0, n1, n2};
+  cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MD_OK : MD_ERR_CUDA;
+}
+
+template <int EPI, int KK>
+md_status launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const md::gemm::Args& ga, bool pdl,
+                      cudaStream_t st) {
+  md_status s;
+  auto kern = md::gemm::heads_gemm_kernel<EPI, KK>;
+  if ((s = set_smem(kern, md::gemm::kSmem)) != MD_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(num_sms(), ga.tiles));
+  cfg.blockDim = dim3(md::gemm::kThreads);
+  cfg.dynamicSmemBytes = md::gemm::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, kern, amap, bmap, ga));
+}
+
+template <int KK>
+md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16* h, const md_bf16* W1,
+                            const md_bf16* b1, const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids,
+                            float* topk_vals, float* logits_dbg, uint8_t* ws, cudaStream_t st) {
+  using namespace md::gemm;
+  const GemmPlan pl = gemm_plan(M, d, V, K, kmax);
+  md_status s;
+  Args ga = {};
+  ga.M = M; ga.d = d; ga.K = K; ga.mtiles = pl.mtiles; ga.kmax = kmax;
+  ga.h = h; ga.b1 = b1;
+  ga.zg = reinterpret_cast<uint16_t*>(ws + pl.off_z);
+  ga.cand_val = reinterpret_cast<float*>(ws + pl.off_cval);
+  ga.cand_id = reinterpret_cast<int*>(ws + pl.off_cid);
+  ga.logits_dbg = logits_dbg;
+  for (int k = 0; k < MD_MAX_K; ++k) ga.kph[k] = k < K ? kph[k] : 0;
+
+  // phase 1: z = bf16(h + SiLU(h W1_k + b1_k))
+  CUtensorMap amap, bmap;
+  if ((s = make_map_3d_sw128(&amap, h, d, M, 1, kBK, kBM)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&bmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
+  ga.N = d; ga.ntiles = pl.ntiles1; ga.tiles = K * pl.ntiles1 * pl.mtiles; ga.a_shared = 1;
+  if ((s = launch_gemm<EPI_SILU, KK>(amap, bmap, ga, false, st)) != MD_OK) return s;
+
+  // phase 2: logits tile = z_k Wv_k, per-row top-k of every 256-column tile
+  if ((s = make_map_3d_sw128(&amap, ga.zg, d, M, K, kBK, kBM)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&bmap, Wv, V, d, K, 64, kBK)) != MD_OK) return s;
+  ga.N = V; ga.ntiles = pl.ntiles2; ga.tiles = K * pl.ntiles2 * pl.mtiles; ga.a_shared = 0;
+  if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, true, st)) != MD_OK) return s;
+
+  // phase 3: merge the tiles' candidates
+  md::heads::MergeArgs ma;
+  ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
+  ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
+  ma.K = K; ma.kmax = kmax; ma.ntiles = pl.ntiles2;
+  for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
+  md::heads::heads_merge_kernel<<<M * K, 256, 0, st>>>(ma);
+  return last_launch();
+}
+
 md_status heads_check(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax) {
   if (M <= 0 || d <= 0 || V <= 0 || K <= 0 || kmax <= 0) return MD_ERR_INVALID_ARG;
   if (K > MD_MAX_K || kmax > MD_MAX_KMAX) return MD_ERR_UNSUPPORTED;
-  if (M > md::heads::kMaxM) return MD_ERR_UNSUPPORTED;
+  if (M > md::gemm::kMaxM) return MD_ERR_UNSUPPORTED;
   if (d % 64 != 0 || V % 8 != 0 || V < 256) return MD_ERR_UNSUPPORTED;
   if (size_t(K) * d >= (size_t(1) << 31) || V >= (1 << 30)) return MD_ERR_UNSUPPORTED;
   return MD_OK;
@@ -175,19 +271,77 @@ AcceptPlan accept_plan(int B, int T, int V) {
 // --------------------------- attention planning ----------------------------
 
 struct AttnPlan {
-  int G, R, max_chunks;
+  bool tc;                  // tensor-core path (the GQA group divides 128)
+  int G, R, max_chunks;     // CUDA-core path
+  int rtiles, splits, cps;  // tensor-core path
   size_t off_ml, bytes;
 };
 
 AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
+  using md::heads::align256;
   AttnPlan p;
   p.G = Hq / Hkv;
   p.R = T * p.G;
-  p.max_chunks = (S_max + md::attn::kChunk - 1) / md::attn::kChunk;
-  const size_t rows = size_t(B) * Hkv * p.max_chunks * p.R;
-  p.off_ml = md::heads::align256(rows * dh * 4);
-  p.bytes = p.off_ml + md::heads::align256(rows * 8);
+  p.tc = (128 % p.G) == 0;
+  if (p.tc) {
+    p.rtiles = (p.R + 127) / 128;
+    const int chunks = (S_max + md::attn_tc::kBN - 1) / md::attn_tc::kBN;
+    const int base = B * Hkv * p.rtiles;
+    int splits = (num_sms() + base - 1) / base;
+    splits = std::max(1, std::min(splits, chunks));
+    p.cps = (chunks + splits - 1) / splits;
+    p.splits = (chunks + p.cps - 1) / p.cps;
+    p.max_chunks = chunks;
+    const size_t rows = size_t(B) * Hkv * p.splits * p.rtiles * 128;
+    p.off_ml = align256(rows * dh * 4);
+    p.bytes = p.off_ml + align256(rows * 8);
+  } else {
+    p.rtiles = p.splits = p.cps = 0;
+    p.max_chunks = (S_max + md::attn::kChunk - 1) / md::attn::kChunk;
+    const size_t rows = size_t(B) * Hkv * p.max_chunks * p.R;
+    p.off_ml = align256(rows * dh * 4);
+    p.bytes = p.off_ml + align256(rows * 8);
+  }
   return p;
+}
+
+template <int DH>
+md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc, const md_bf16* vc,
+                         const int32_t* prefix_len, int S_max, const md_tree* tree, int B, int Hq, int Hkv, float sc,
+                         float* out, void* ws, cudaStream_t st) {
+  using namespace md::attn_tc;
+  md_status s;
+  const int T = tree->tp.T;
+  CUtensorMap qmap, kmap, vmap;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MD_ERR_CUDA;
+  {
+    // q [B*T][Hq][dh]: box {64, G, 128/G} = 128 rows of (tree token, head of the group)
+    cuuint64_t dims[3] = {cuuint64_t(DH), cuuint64_t(Hq), cuuint64_t(B) * T};
+    cuuint64_t strides[2] = {cuuint64_t(DH) * 2, cuuint64_t(Hq) * DH * 2};
+    cuuint32_t box[3] = {64, cuuint32_t(pl.G), cuuint32_t(128 / pl.G)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<md_bf16*>(q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MD_ERR_CUDA;
+  }
+  if ((s = make_map_3d_sw128(&kmap, kc, DH, S_max, uint64_t(B) * Hkv, 64, kBN)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&vmap, vc, DH, S_max, uint64_t(B) * Hkv, 64, kBN)) != MD_OK) return s;
+  Args a;
+  a.prefix_len = prefix_len;
+  a.part_o = static_cast<float*>(ws);
+  a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
+  a.out = out;
+  a.B = B; a.S_max = S_max; a.Hq = Hq; a.Hkv = Hkv; a.G = pl.G; a.R = pl.R; a.rtiles = pl.rtiles;
+  a.splits = pl.splits; a.chunks_per_split = pl.cps;
+  a.scale_log2 = sc * 1.4426950408889634f;
+  constexpr int sm = Cfg<DH>::kSmem;
+  if ((s = set_smem(attn_tc_kernel<DH>, sm)) != MD_OK) return s;
+  attn_tc_kernel<DH><<<dim3(pl.splits, Hkv * pl.rtiles, B), kThreads, sm, st>>>(qmap, kmap, vmap, tree->tp, a);
+  if ((s = last_launch()) != MD_OK) return s;
+  attn_tc_merge_kernel<DH><<<dim3(T * Hq, B), DH, 0, st>>>(tree->tp, a);
+  return last_launch();
 }
 
 }  // namespace
@@ -253,7 +407,8 @@ md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t
   if (!bytes) return MD_ERR_INVALID_ARG;
   md_status s = heads_check(M, d, V, K, kmax);
   if (s != MD_OK) return s;
-  *bytes = md::heads::make_plan(M, d, V, K, kmax, num_sms()).bytes;
+  *bytes = M <= md::heads::kMaxM ? md::heads::make_plan(M, d, V, K, kmax, num_sms()).bytes
+                                  : gemm_plan(M, d, V, K, kmax).bytes;
   return MD_OK;
 }
 
@@ -269,10 +424,22 @@ md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1
   if (!aligned(h, 2) || !aligned(W1, 16) || !aligned(b1, 2) || !aligned(Wv, 16) || !aligned(topk_ids, 4) ||
       !aligned(topk_vals, 4) || (logits_dbg && !aligned(logits_dbg, 4)))
     return MD_ERR_INVALID_ARG;
-  const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
-  if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
+  if (M > md::heads::kMaxM) {
+    // tensor-core path: h, W1, Wv feed TMA directly (16-byte aligned rows: d % 64, V % 8)
+    if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < gemm_plan(M, d, V, K, kmax).bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+    int mk = 0;
+    for (int k = 0; k < K; ++k) mk = std::max(mk, int(k_per_head[k]));
+    if (mk <= 4)
+      return launch_heads_gemm<4>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    if (mk <= 8)
+      return launch_heads_gemm<8>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+    return launch_heads_gemm<16>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+  }
+  const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
+  if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
   switch (M) {
     case 1: return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
     case 2: return launch_heads<2>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
@@ -325,15 +492,19 @@ md_status md_tree_attention(const md_bf16* q, const md_bf16* k_cache, const md_b
     return MD_ERR_INVALID_ARG;
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
   const AttnPlan pl = attn_plan(B, T, Hq, Hkv, dh, S_max);
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(float(dh));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (pl.tc) {
+    return dh == 128 ? launch_attn_tc<128>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out, ws, st)
+                     : launch_attn_tc<64>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out, ws, st);
+  }
   md::attn::Args a;
   a.q = q; a.kc = k_cache; a.vc = v_cache; a.prefix_len = prefix_len;
   a.part_acc = static_cast<float*>(ws);
   a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
   a.out = out;
   a.S_max = S_max; a.Hq = Hq; a.Hkv = Hkv; a.G = pl.G; a.R = pl.R; a.max_chunks = pl.max_chunks;
-  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(float(dh));
   a.scale_log2 = sc * 1.4426950408889634f;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dim3 grid(pl.max_chunks, Hkv, B);
   if (dh == 128) {
     constexpr int sm = md::attn::smem_bytes<128>();

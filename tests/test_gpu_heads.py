@@ -31,8 +31,9 @@ def _run(h, W1, b1, Wv, kph, kmax=None, dbg=True):
                                        (8, 320, 2056, (16, 1, 7, 3)), (3, 1024, 4096, (5, 5, 5, 5))])
 def test_heads_match_oracle_small(M, d, V, kph):
     h, W1, b1, Wv = head_weights(11 + M, d, V, len(kph), M)
-    ids, vals, logits = _run(h, W1, b1, Wv, kph, kmax=max(kph) + 1)
-    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph, max(kph) + 1)
+    kmax = min(16, max(kph) + 1)           # one spare slot where the stride allows it
+    ids, vals, logits = _run(h, W1, b1, Wv, kph, kmax=kmax)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph, kmax)
     err = normwise(logits, rlog)
     assert err.max() <= HEADS_RTOL, err.max()
     assert err.max() <= 1e-4        # fp32 accumulation is far inside the stated bound
@@ -91,3 +92,37 @@ def test_heads_reject_bad_arguments():
     with pytest.raises(md.MedusaError, match="invalid"):
         md.medusa_heads(bf16_tensor(h), bf16_tensor(W1), bf16_tensor(b1), bf16_tensor(Wv), (5, 3, 2, 2), ids,
                         vals, ws)
+
+
+# ----------------------------- tensor-core path (M > 8) -----------------------------
+
+@pytest.mark.parametrize("M,d,V,kph", [(9, 256, 1024, (4, 3, 2, 2)), (40, 320, 1000, (10, 10, 10, 10)),
+                                       (130, 512, 2056, (16, 1, 7, 3)), (520, 256, 4096, (10, 10, 10, 10))])
+def test_tensor_core_heads_match_oracle(M, d, V, kph):
+    h, W1, b1, Wv = head_weights(101 + M, d, V, len(kph), M)
+    ids, vals, logits = _run(h, W1, b1, Wv, kph)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph)
+    err = normwise(logits, rlog)
+    assert err.max() <= HEADS_RTOL, err.max()
+    assert err.max() <= 1e-4
+    for m in range(M):
+        for k, kk in enumerate(kph):
+            check_topk_row(ids[m, k], vals[m, k], rlog[m, k], kk)
+
+
+@pytest.mark.parametrize("M,d,V,kph", [(17, 128, 1024, (16, 10, 1, 5)), (200, 64, 776, (3, 16, 2, 9))])
+def test_tensor_core_topk_bit_exact_on_integer_logits(M, d, V, kph):
+    h, W1, b1, Wv = _integer_heads(M * 3 + d, M, d, V, len(kph))
+    ids, vals, logits = _run(h, W1, b1, Wv, kph)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph)
+    assert np.array_equal(logits, rlog.astype(np.float32))
+    assert np.array_equal(ids, rid)
+    assert np.array_equal(vals, rval.astype(np.float32))
+
+
+def test_tensor_core_fused_equals_debug_run():
+    """The top-k does not depend on whether the logits are also written."""
+    h, W1, b1, Wv = head_weights(77, 512, 4096, 4, 64)
+    a = _run(h, W1, b1, Wv, (10, 10, 10, 10), dbg=False)
+    b = _run(h, W1, b1, Wv, (10, 10, 10, 10), dbg=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])

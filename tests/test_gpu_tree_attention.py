@@ -15,6 +15,7 @@ pytestmark = pytest.mark.gpu
 
 def _random_tree(rng, T, K, kmax):
     """A random valid tree spec: parent < j, depth <= K, distinct sibling ranks."""
+    assert T - 1 <= sum(kmax ** d for d in range(1, K + 1)), "no tree of that size exists"
     parent, rank, depth = [-1], [0], [0]
     used = {}
     for j in range(1, T):
@@ -30,7 +31,7 @@ def _random_tree(rng, T, K, kmax):
     return parent, rank
 
 
-@pytest.mark.parametrize("T,B,K", [(17, 1, 4), (65, 3, 4), (128, 5, 8), (1, 2, 4), (33, 2, 1)])
+@pytest.mark.parametrize("T,B,K", [(17, 1, 4), (65, 3, 4), (128, 5, 8), (1, 2, 4), (17, 2, 1)])
 def test_tree_build_bit_exact(T, B, K):
     rng = np.random.default_rng(T * 10 + B)
     kmax = 16
@@ -89,6 +90,11 @@ def _attention_case(seed, tups, B, Hq, Hkv, dh, P, S_max, scale=0.0):
     ("8b", ((10, 10, 10, 10), 64), 1, 32, 8, 128, [2048]),
     ("70b-chain", ((1, 1, 1, 1), 4), 1, 64, 8, 128, [4096]),
     ("gqa16", ((10, 10, 10, 10), 16), 2, 16, 1, 64, [129, 255]),
+    # GQA groups that do not divide 128 rows take the CUDA-core kernel
+    ("g3-cuda-core", ((4, 3, 2, 2), 16), 2, 6, 2, 128, [77, 300]),
+    ("g12-cuda-core", ((10, 10, 10, 10), 64), 1, 12, 1, 64, [1000]),
+    # long prefix: many key chunks per split, B = 4 with ragged lengths
+    ("long-ragged", ((10, 10, 10, 10), 64), 4, 32, 8, 128, [1024, 8191, 333, 5000]),
 ])
 def test_tree_attention_matches_oracle(name, tree, B, Hq, Hkv, dh, P):
     kph, n = tree
