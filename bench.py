@@ -52,12 +52,12 @@ def heads_bytes(w):
 
 
 def attention_bytes(w, P):
-    kv = sum(2 * w.Hkv * (p + w.T) * w.dh * 2 for p in P)
+    kv = sum(2 * w.Hkv * (int(p) + w.T) * w.dh * 2 for p in P)
     return kv + w.B * w.T * w.Hq * w.dh * (2 + 4)
 
 
 def attention_flops(w, P):
-    return sum(4 * w.Hq * w.T * (p + w.T) * w.dh for p in P)
+    return sum(4 * w.Hq * w.T * (int(p) + w.T) * w.dh for p in P)
 
 
 def accept_bytes(w):

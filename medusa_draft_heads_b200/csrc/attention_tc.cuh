@@ -15,9 +15,10 @@
 //              and O_c = P_c V_c into TMEM
 //   warps 2-5  one query row per thread: read S_c from TMEM, apply the scale
 //              and the tree mask (keys >= P_b are tree nodes; visible iff an
-//              ancestor-or-self), chunk max, P_c = exp2(S - max) rounded to
-//              bf16 into swizzled shared memory, and fold O_{c-1} into a
-//              running (max, sum, O) kept in registers.
+//              ancestor-or-self), chunk max, P_c = exp2(S - max) split into
+//              bf16 hi + lo parts in swizzled shared memory (P V then runs as
+//              P_hi V + P_lo V, so the weights keep ~16 significant bits), and
+//              fold O_{c-1} into a running (max, sum, O) kept in registers.
 //
 // Each CTA writes its split's (max, sum, unnormalised O) per row;
 // attn_tc_merge_kernel combines the splits in order.
@@ -41,7 +42,7 @@ struct Cfg {
   static constexpr uint32_t kVBytes = KB * kBN * 128;         // V chunk, N(dh)-major SW128
   static constexpr uint32_t kStage = kKBytes + kVBytes;
   static constexpr uint32_t kPBytes = 2 * kBM * 128;          // P tile: 128 rows x 128 keys bf16
-  static constexpr int kSmem = kQBytes + 2 * kStage + kPBytes + 1024 + 256;
+  static constexpr int kSmem = kQBytes + 2 * kStage + 2 * kPBytes + 1024 + 256;   // P hi and P lo
 };
 
 struct Args {
@@ -66,8 +67,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;                     // 2 stages of (K, V)
-  uint8_t* sP = sKV + 2 * C::kStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::kPBytes);
+  uint8_t* sP = sKV + 2 * C::kStage;                    // P hi
+  uint8_t* sPl = sP + C::kPBytes;                        // P lo
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sPl + C::kPBytes);
   uint64_t* q_full = bars;            // 1
   uint64_t* kv_full = bars + 1;       // 2
   uint64_t* kv_empty = bars + 3;      // 2
@@ -179,12 +181,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(smem_u32(p_full), cp & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sv = smem_u32(sKV + (cp & 1) * C::kStage + C::kKBytes);
-          const uint32_t sp = smem_u32(sP);
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t ad = umma_desc_sw128(sp + (kk >> 2) * kBM * 128, 16, 1024) + uint64_t(((kk & 3) * 32) >> 4);
-            const uint64_t bd = umma_desc_sw128(sv, kBN * 128, 1024) + uint64_t((kk * 2048) >> 4);
-            umma_f16(tO, ad, bd, idesc_o, kk != 0);
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t sp = smem_u32(part == 0 ? sP : sPl);
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              const uint64_t ad =
+                  umma_desc_sw128(sp + (kk >> 2) * kBM * 128, 16, 1024) + uint64_t(((kk & 3) * 32) >> 4);
+              const uint64_t bd = umma_desc_sw128(sv, kBN * 128, 1024) + uint64_t((kk * 2048) >> 4);
+              umma_f16(tO, ad, bd, idesc_o, (part | kk) != 0);
+            }
           }
           umma_commit(smem_u32(o_full));
           umma_commit(smem_u32(&kv_empty[cp & 1]));
@@ -247,15 +253,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         fold(cm, cl);
       }
-      // pass 2: P = exp2(S - max) into swizzled smem (K-major over keys)
+      // pass 2: P = exp2(S - max) as bf16 hi + lo into swizzled smem (K-major over keys)
       float sum = 0.f;
       for (int c32 = 0; c32 < kBN; c32 += 32) {
         float s[32];
         tmem_ld32(sb + c32, s);
-        uint32_t pk[16];
+        uint32_t ph[16], pl[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          float p2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int slot = key0 + c32 + j + u;
@@ -265,19 +270,27 @@ __global__ void __launch_bounds__(kThreads, 1)
               vis = live && ((tp.anc[t < T ? t : 0][node >> 5] >> (node & 31)) & 1u);
             }
             const float p = (vis && mx != -INFINITY) ? exp2f(s[j + u] * a.scale_log2 - mx) : 0.f;
-            const uint16_t pb = f32_to_bf16_rne(p);
-            p2[u] = bf16_to_f32(pb);   // the sum uses the rounded weights the MMA sees
-            sum += p2[u];
-            if (u == 0) pk[j >> 1] = pb; else pk[j >> 1] |= uint32_t(pb) << 16;
+            const uint16_t hb = f32_to_bf16_rne(p);
+            const float hf = bf16_to_f32(hb);
+            const uint16_t lb = f32_to_bf16_rne(p - hf);
+            sum += hf + bf16_to_f32(lb);   // the weights the two MMAs apply
+            if (u == 0) {
+              ph[j >> 1] = hb;
+              pl[j >> 1] = lb;
+            } else {
+              ph[j >> 1] |= uint32_t(hb) << 16;
+              pl[j >> 1] |= uint32_t(lb) << 16;
+            }
           }
         }
         // row r, keys c32 .. c32+31 -> block c32/64, 16-byte chunks (c32%64)/8 .. +3, swizzled by r%8
-        uint8_t* rowp = sP + (c32 >> 6) * kBM * 128 + r * 128;
+        const uint32_t roff = (c32 >> 6) * kBM * 128 + r * 128;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int ch = ((c32 & 63) >> 3) + g;
-          *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+          const uint32_t off = roff + ((ch ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(sP + off) = make_uint4(ph[4 * g], ph[4 * g + 1], ph[4 * g + 2], ph[4 * g + 3]);
+          *reinterpret_cast<uint4*>(sPl + off) = make_uint4(pl[4 * g], pl[4 * g + 1], pl[4 * g + 2], pl[4 * g + 3]);
         }
       }
       cm = mx;
