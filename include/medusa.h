@@ -144,6 +144,40 @@ MD_API md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_b
                           int32_t kmax, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the library-owned scratch behind md_medusa_heads_static (8 MiB). */
+#define MD_HEADS_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* md_medusa_heads for callers that cannot allocate device memory.
+ * (An addition of this library: the pages have no counterpart.)
+ *
+ * Some callers have no way to hand the library a workspace: code that runs
+ * while a CUDA graph is being captured (where cudaMalloc is not allowed),
+ * runtimes whose device memory is fully owned by a pool that no plugin may
+ * grow, or hot loops that must never reach the allocator. This entry point
+ * computes exactly what md_medusa_heads computes, with the same arguments
+ * minus the workspace: its scratch is a fixed MD_HEADS_STATIC_SCRATCH_BYTES
+ * array inside the library's device image, which every GPU that loads the
+ * library keeps until the process exits. It calls no cudaMalloc, cudaFree or
+ * other allocating routine. The caller still provides the inputs and outputs.
+ *
+ * - Sizes whose scratch (md_heads_workspace) exceeds the array are rejected
+ *   with MD_ERR_WORKSPACE before anything is launched (at d = 8192,
+ *   V = 128256, K = 4, kmax = 10 this admits M <= 6, and M = 9 .. 37 on the
+ *   tensor-core path).
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture on the device.
+ * - Every call on a device shares the one array and leaves its contents
+ *   behind; the call clears what must start at zero itself. Two calls whose
+ *   kernels overlap on the GPU (different streams, no ordering between them)
+ *   race on the array and give undefined results: order them on one stream
+ *   or with events.
+ * Errors: as md_medusa_heads, plus MD_ERR_WORKSPACE for oversized shapes. */
+MD_API md_status md_medusa_heads_static(const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
+                                        const md_bf16* Wv, int32_t M, int32_t d, int32_t V, int32_t K,
+                                        const int32_t* k_per_head, int32_t kmax, int32_t* topk_ids,
+                                        float* topk_vals, float* logits_dbg, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* 2. Candidate tree construction.                                           */
 /* ------------------------------------------------------------------------ */

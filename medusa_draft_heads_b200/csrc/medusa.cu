@@ -4,6 +4,7 @@
 // single module-scope variable without relocatable device code.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "common.cuh"
@@ -344,6 +345,32 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   return last_launch();
 }
 
+// Scratch of md_medusa_heads_static: a fixed array in the library's device
+// image (every GPU that loads the library holds it until the process exits).
+__device__ __align__(256) uint8_t g_heads_static_scratch[MD_HEADS_STATIC_SCRATCH_BYTES];
+
+// Device address of g_heads_static_scratch on the current device. Host code
+// cannot use the symbol itself (on the host it names a stand-in, not device
+// memory), so the address is looked up once per device, with that device
+// current, and cached.
+md_status static_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MD_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_heads_static_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return MD_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return MD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -451,6 +478,19 @@ md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1
     case 8: return launch_heads<8>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
     default: return MD_ERR_UNSUPPORTED;
   }
+}
+
+md_status md_medusa_heads_static(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
+                                 int32_t M, int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax,
+                                 int32_t* topk_ids, float* topk_vals, float* logits_dbg, void* stream) {
+  size_t need = 0;
+  md_status s = md_heads_workspace(M, d, V, K, kmax, &need);
+  if (s != MD_OK) return s;
+  if (need > size_t(MD_HEADS_STATIC_SCRATCH_BYTES)) return MD_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != MD_OK) return s;
+  return md_medusa_heads(h, W1, b1, Wv, M, d, V, K, k_per_head, kmax, topk_ids, topk_vals, logits_dbg, scratch,
+                         size_t(MD_HEADS_STATIC_SCRATCH_BYTES), stream);
 }
 
 md_status md_tree_build(const md_tree* tree, const int32_t* topk_ids, int32_t M, int32_t kmax,
