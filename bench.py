@@ -398,6 +398,71 @@ def run_medusa(args, w):
         dist.destroy_process_group()
 
 
+def run_part(args, w):
+    """Time one of the four calls alone on the workload's shapes (for profiling
+    and per-kernel study); only that call's inputs are allocated."""
+    import torch
+
+    import medusa_draft_heads_b200 as md
+    from medusa_draft_heads_b200.step import MedusaStep
+    from seeded_inputs import device as sdev
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    seed = w.seed
+    tups = md.select_tree(w.k_per_head, w.accept, w.n_nodes)
+    step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
+                      Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
+                      alpha=w.alpha, device=dev)
+    P = synth.prefix_lengths(seed, w.B, *w.prefix)
+    prefix = torch.from_numpy(P).to(dev)
+    if args.part == "heads":
+        W1 = sdev.fill_normal(torch.empty((w.K, w.d, w.d), **bf), seed, "W1", w.w_sigma)
+        b1 = sdev.fill_normal(torch.empty((w.K, w.d), **bf), seed, "b1", w.w_sigma)
+        Wv = sdev.fill_normal(torch.empty((w.K, w.d, w.V), **bf), seed, "Wv", w.w_sigma)
+        h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), seed, "h", 1.0)
+        call = lambda i: step.heads(h, W1, b1, Wv)                              # noqa: E731
+        nbytes, nflops, launches = heads_bytes(w), 2 * w.M * w.K * w.d * (w.d + w.V), 3
+    elif args.part == "attention":
+        nsets = 8
+        sets = [(sdev.fill_normal(torch.empty((w.B, w.T, w.Hq, w.dh), **bf), seed + i, "q", 1.0),
+                 sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + i, "k_cache", 1.0),
+                 sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + i, "v_cache", 1.0))
+                for i in range(nsets)]
+        call = lambda i: step.attention(*sets[i % nsets], prefix)                # noqa: E731
+        nbytes, nflops, launches = attention_bytes(w, P), attention_flops(w, P), 2
+    else:
+        tokens = synth.synthetic_tree_tokens(seed, w.B, np.array(step.tree.parent), w.V)
+        logits = synth.planted_logits(seed, np.array(step.tree.parent), tokens, w.V, w.accept,
+                                      sigma=w.logit_sigma, bump=w.bump)
+        step.tokens.copy_(torch.from_numpy(tokens))
+        nsets = max(2, -(-2 * L2_BYTES // logits.nbytes))
+        lgs = [torch.from_numpy(logits).to(dev) for _ in range(nsets)]
+        call = lambda i: step.accept(lgs[i % nsets])                              # noqa: E731
+        nbytes, nflops, launches = accept_bytes(w), 0, 2
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            call(i)
+    stream.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            call(i)
+        end.record(stream)
+    torch.cuda.synchronize()
+    status = md.device_status(stream=stream)
+    ms = start.elapsed_time(end) / args.steps
+    peaks = measured_peaks()
+    print(json.dumps({"part": args.part, "workload": w.name, "ms_per_call": ms, "calls": args.steps,
+                      "gbs": nbytes / (ms / 1000) / 1e9, "hbm_frac": nbytes / (ms / 1000) / 1e9 / peaks["hbm_gbs"],
+                      "tflops": nflops / (ms / 1000) / 1e12 if nflops else None,
+                      "algorithmic_bytes": nbytes, "flops": nflops, "gpu_launches": launches * args.steps,
+                      "device_status": status}), flush=True)
+
+
 def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, dev, world, barrier):
     """Same step through the public API, with this step's inputs copied from
     pinned host memory and the result read back every step."""
@@ -479,6 +544,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["medusa", "reference"], default="medusa")
     ap.add_argument("--workload", default="llama3-70b", choices=sorted(WORKLOADS))
+    ap.add_argument("--part", choices=["step", "heads", "attention", "accept"], default="step",
+                    help="time one call alone (profiling); the JSON line then reports that call only")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-frac", type=float, default=1 / 64)
@@ -490,6 +557,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.part != "step":
+        run_part(args, w)
+        return
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return

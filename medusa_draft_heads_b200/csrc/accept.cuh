@@ -78,16 +78,30 @@ __global__ void __launch_bounds__(kRowThreads) accept_rows_kernel(Args a) {
   int bi = INT_MAX;
   Soft sm{-INFINITY, 0.f, 0.f};
   const bool typical = a.mode == MD_ACCEPT_TYPICAL;
-  for (int v = v0 + threadIdx.x * 4; v < v1; v += kRowThreads * 4) {
-    const float4 f = ld_stream_f4(x + v);
-    const float fv[4] = {f.x, f.y, f.z, f.w};
+  // kUnroll independent 16-byte loads in flight per thread before any use.
+  constexpr int kUnroll = 8;
+  constexpr int kStep = kRowThreads * 4;
+  for (int base = v0 + threadIdx.x * 4; base < v1; base += kStep * kUnroll) {
+    float4 f[kUnroll];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (better(fv[e], v + e, bv, bi)) {
-        bv = fv[e];
-        bi = v + e;
+    for (int u = 0; u < kUnroll; ++u) {
+      const int v = base + u * kStep;
+      f[u] = v < v1 ? ld_stream_f4(x + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int v = base + u * kStep;
+      if (v < v1) {
+        const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (better(fv[e], v + e, bv, bi)) {
+            bv = fv[e];
+            bi = v + e;
+          }
+          if (typical) soft_add(sm, fv[e] * a.inv_temp);
+        }
       }
-      if (typical) soft_add(sm, fv[e] * a.inv_temp);
     }
   }
   // Block reduction (fixed shuffle tree, then warps in order).

@@ -13,6 +13,8 @@
 //   phase 3  heads_merge_kernel    top-k over every tile's candidates
 #pragma once
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace md {
@@ -38,6 +40,7 @@ struct Plan {
   int ntiles;   // phase-2 vocabulary tiles
   int units;    // K * ntiles
   int nstages;  // phase-2 pipeline depth
+  int grid;     // phase-2 CTAs (one candidate list per row, head and CTA)
   size_t off_zt, off_part, off_cnt, off_cval, off_cid, bytes;
 };
 
@@ -67,8 +70,9 @@ inline Plan make_plan(int M, int d, int V, int K, int kmax, int num_sms) {
   p.off_zt = o;   o = align256(o + size_t(K) * d * kZPad * 2);
   p.off_part = o; o = align256(o + size_t(splits) * K * M * d * 4);
   p.off_cnt = o;  o = align256(o + size_t(K) * p.ntile_o * 4);
-  p.off_cval = o; o = align256(o + size_t(M) * K * p.ntiles * kmax * 4);
-  p.off_cid = o;  o = align256(o + size_t(M) * K * p.ntiles * kmax * 4);
+  p.grid = std::min(num_sms, p.units);
+  p.off_cval = o; o = align256(o + size_t(M) * K * p.grid * kmax * 4);
+  p.off_cid = o;  o = align256(o + size_t(M) * K * p.grid * kmax * 4);
   p.bytes = o;
   return p;
 }
@@ -213,17 +217,19 @@ __global__ void __launch_bounds__(kW1Threads) heads_w1_kernel(W1Args a) {
 }
 
 // ---------------------------------------------------------------------------
-// Phase 2: persistent vocabulary stream with the per-tile top-k fused in.
+// Phase 2: persistent vocabulary stream with the top-k fused in.
 // grid = min(#SMs, K * ntiles), 288 threads: warps 0..7 do the math, warp 8
 // issues the TMA loads. A work unit is (head k, 256-column tile); it walks
 // d / 64 stages of [64 rows x 256 cols] of Wv_k plus the matching 64 rows of
-// z_k. Warp w multiplies rows 8w..8w+7 of each stage, lane l columns
-// 8l..8l+7, fp32 accumulate; the eight warps' partials are summed in fixed
-// order, then warp m picks the tile's top-k of row m.
+// z_k. CTA c owns the contiguous units [c*U/G, (c+1)*U/G). Warp w multiplies
+// rows 8w..8w+7 of each stage, lane l columns 8l..8l+7, fp32 accumulate; the
+// eight warps' partials are summed in fixed order, then warp m folds the
+// tile's 256 logits of row m into a running top-k of (row m, head k), which
+// is written out once per (CTA, head): one candidate list per CTA and head.
 // ---------------------------------------------------------------------------
 struct VocabArgs {
   const uint16_t* zt;  // [K, d, 8]
-  float* cand_val;     // [M, K, ntiles, kmax]
+  float* cand_val;     // [M, K, gridDim.x, kmax]: one list per (row, head, CTA)
   int* cand_id;
   float* logits_dbg;   // [M, K, V] or null
   int d, V, K, kmax, ntiles, units, nstages;
@@ -263,7 +269,9 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       bool waited_primary = false;
       int it = 0;
       bool ok = true;
-      for (int unit = blockIdx.x; unit < a.units && ok; unit += gridDim.x) {
+      const int u0 = int((long long)blockIdx.x * a.units / gridDim.x);
+      const int u1 = int((long long)(blockIdx.x + 1) * a.units / gridDim.x);
+      for (int unit = u0; unit < u1 && ok; ++unit) {
         const int k = unit / a.ntiles, tile = unit % a.ntiles;
         for (int s = 0; s < stages_per_unit; ++s, ++it) {
           const int slot = it % ns;
@@ -299,7 +307,12 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
   // -------------------------------- consumers --------------------------------
   int it = 0;
   bool ok = true;
-  for (int unit = blockIdx.x; unit < a.units; unit += gridDim.x) {
+  const int u0 = int((long long)blockIdx.x * a.units / gridDim.x);
+  const int u1 = int((long long)(blockIdx.x + 1) * a.units / gridDim.x);
+  // Running top-k of (row m = warp, current head): lane r holds entry r.
+  float rv = -INFINITY;
+  int ri = INT_MAX;
+  for (int unit = u0; unit < u1; ++unit) {
     const int k = unit / a.ntiles, tile = unit % a.ntiles;
     float acc[M][8];
 #pragma unroll
@@ -363,8 +376,9 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
     }
     named_bar_sync(1, kConsumerWarps * 32);
 
-    // Per-tile top-k of row m by warp m: k rounds, each taking the best entry
-    // strictly after the previous winner in (value desc, id asc) order.
+    // Warp m folds the tile into its running top-k: k rounds, each taking the
+    // best entry strictly after the previous winner in (value desc, id asc)
+    // order among the tile's 256 logits and the running list.
     if (warp < M) {
       const int m = warp;
       float v[kTileV / 32];
@@ -378,7 +392,8 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       float pv = INFINITY;
       int pid = -1;
       const int kk = a.kph[k];
-      const size_t cbase = ((size_t(m) * a.K + k) * a.ntiles + tile) * a.kmax;
+      float nrv = -INFINITY;
+      int nri = INT_MAX;
       for (int r = 0; r < kk; ++r) {
         float bv = -INFINITY;
         int bi = INT_MAX;
@@ -389,6 +404,10 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
             bi = id[i];
           }
         }
+        if (better(pv, pid, rv, ri) && better(rv, ri, bv, bi)) {
+          bv = rv;
+          bi = ri;
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
           const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
@@ -398,57 +417,90 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
             bi = oi;
           }
         }
-        if (lane == 0) {
-          a.cand_val[cbase + r] = bv;
-          a.cand_id[cbase + r] = (bi == INT_MAX) ? -1 : bi;
+        if (lane == r) {
+          nrv = bv;
+          nri = bi;
         }
         pv = bv;
         pid = bi;
+      }
+      rv = nrv;
+      ri = nri;
+      // flush the list when the next unit belongs to another head (or there is none)
+      if (unit + 1 == u1 || (unit + 1) / a.ntiles != k) {
+        if (lane < kk) {
+          const size_t cb = ((size_t(m) * a.K + k) * gridDim.x + blockIdx.x) * a.kmax + lane;
+          a.cand_val[cb] = rv;
+          a.cand_id[cb] = (ri == INT_MAX) ? -1 : ri;
+        }
+        rv = -INFINITY;
+        ri = INT_MAX;
       }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Phase 3: merge the tiles' candidates into each head's top-k.
-// grid (M * K), 256 threads; k rounds of a block-wide "best entry strictly
-// after the previous winner" reduction.
+// Phase 3: merge candidate lists into each head's top-k.
+// grid (M * K), 256 threads. The candidates of (m, k) are `nslots` lists of
+// up to kmax entries. In "partitioned" mode slot c is CTA c of the vocabulary
+// kernel and only CTAs whose unit range touches head k wrote a list. Each
+// thread gathers its slots into a sorted register list; each warp then merges
+// its 32 lists by k rounds of a shuffle arg-max over the list heads (the
+// winning lane shifts its list), and warp 0 merges the 8 warp lists the same way.
 // ---------------------------------------------------------------------------
 struct MergeArgs {
   const float* cand_val;
   const int* cand_id;
   int32_t* topk_ids;   // [M, K, kmax]
   float* topk_vals;
-  int K, kmax, ntiles;
+  int K, kmax, nslots;
+  int partitioned, units, ntiles;   // vocabulary-kernel partition (partitioned == 1)
   int kph[MD_MAX_K];
 };
 
-__global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
-  __shared__ float sv[8];
-  __shared__ int si[8];
-  __shared__ float wv;
-  __shared__ int wi;
-  const int mk = blockIdx.x;
-  const int k = mk % a.K;
-  const int kk = a.kph[k];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t base = size_t(mk) * a.ntiles * a.kmax;
-  const int n = a.ntiles * kk;
-  float pv = INFINITY;
-  int pid = -1;
-  for (int r = 0; r < kk; ++r) {
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-    for (int idx = threadIdx.x; idx < n; idx += 256) {
-      const int tile = idx / kk, j = idx - tile * kk;
-      const float cv = a.cand_val[base + size_t(tile) * a.kmax + j];
-      int ci = a.cand_id[base + size_t(tile) * a.kmax + j];
-      if (ci < 0) ci = INT_MAX;
-      if (better(pv, pid, cv, ci) && better(cv, ci, bv, bi)) {
-        bv = cv;
-        bi = ci;
+constexpr int kListMax = MD_MAX_KMAX;
+
+struct SortedList {
+  float v[kListMax];
+  int i[kListMax];
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int j = 0; j < kListMax; ++j) {
+      v[j] = -INFINITY;
+      i[j] = INT_MAX;
+    }
+  }
+  __device__ __forceinline__ void push(float x, int id) {
+    if (!better(x, id, v[kListMax - 1], i[kListMax - 1])) return;
+    v[kListMax - 1] = x;
+    i[kListMax - 1] = id;
+#pragma unroll
+    for (int j = kListMax - 1; j > 0; --j) {
+      if (better(v[j], i[j], v[j - 1], i[j - 1])) {
+        const float tv = v[j]; v[j] = v[j - 1]; v[j - 1] = tv;
+        const int ti = i[j]; i[j] = i[j - 1]; i[j - 1] = ti;
       }
     }
+  }
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int j = 0; j < kListMax - 1; ++j) {
+      v[j] = v[j + 1];
+      i[j] = i[j + 1];
+    }
+    v[kListMax - 1] = -INFINITY;
+    i[kListMax - 1] = INT_MAX;
+  }
+};
+
+// kk rounds over the warp's lists; round r's winner is returned to lane r.
+__device__ __forceinline__ void warp_merge(SortedList& L, int kk, int lane, float& out_v, int& out_i) {
+  out_v = -INFINITY;
+  out_i = INT_MAX;
+  for (int r = 0; r < kk; ++r) {
+    float bv = L.v[0];
+    int bi = L.i[0];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
@@ -458,37 +510,54 @@ __global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
         bi = oi;
       }
     }
-    if (lane == 0) {
-      sv[warp] = bv;
-      si[warp] = bi;
+    if (bi != INT_MAX && L.i[0] == bi && L.v[0] == bv) L.pop();
+    if (lane == r) {
+      out_v = bv;
+      out_i = bi;
     }
-    __syncthreads();
-    if (warp == 0) {
-      bv = lane < 8 ? sv[lane] : -INFINITY;
-      bi = lane < 8 ? si[lane] : INT_MAX;
-#pragma unroll
-      for (int off = 4; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (lane == 0) {
-        wv = bv;
-        wi = bi;
-        a.topk_vals[size_t(mk) * a.kmax + r] = bv;
-        a.topk_ids[size_t(mk) * a.kmax + r] = (bi == INT_MAX) ? -1 : bi;
-      }
-    }
-    __syncthreads();
-    pv = wv;
-    pid = wi;
   }
-  for (int r = kk + threadIdx.x; r < a.kmax; r += 256) {
-    a.topk_vals[size_t(mk) * a.kmax + r] = -INFINITY;
-    a.topk_ids[size_t(mk) * a.kmax + r] = -1;
+}
+
+__global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
+  __shared__ float wv[8][kListMax];
+  __shared__ int wi[8][kListMax];
+  const int mk = blockIdx.x;
+  const int k = mk % a.K;
+  const int kk = a.kph[k];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t base = size_t(mk) * a.nslots * a.kmax;
+  SortedList L;
+  L.clear();
+  for (int c = threadIdx.x; c < a.nslots; c += 256) {
+    if (a.partitioned) {
+      const long long u0 = (long long)c * a.units / a.nslots, u1 = (long long)(c + 1) * a.units / a.nslots;
+      if (u1 <= (long long)k * a.ntiles || u0 >= (long long)(k + 1) * a.ntiles) continue;
+    }
+    for (int j = 0; j < kk; ++j) {
+      const int id = a.cand_id[base + size_t(c) * a.kmax + j];
+      if (id >= 0) L.push(a.cand_val[base + size_t(c) * a.kmax + j], id);
+    }
+  }
+  float ov;
+  int oi;
+  warp_merge(L, kk, lane, ov, oi);
+  if (lane < kk) {
+    wv[warp][lane] = ov;
+    wi[warp][lane] = oi;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    L.clear();
+    if (lane < 8) {
+      for (int j = 0; j < kk; ++j)
+        if (wi[lane][j] != INT_MAX) L.push(wv[lane][j], wi[lane][j]);
+    }
+    warp_merge(L, kk, lane, ov, oi);
+    if (lane < a.kmax) {
+      const bool used = lane < kk && oi != INT_MAX;
+      a.topk_vals[size_t(mk) * a.kmax + lane] = used ? ov : -INFINITY;
+      a.topk_ids[size_t(mk) * a.kmax + lane] = used ? oi : -1;
+    }
   }
 }
 

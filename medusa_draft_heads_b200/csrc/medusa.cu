@@ -124,7 +124,7 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   const int v_smem = vocab_smem_bytes(M, pl.nstages);
   if ((s = set_smem(heads_vocab_kernel<M>, v_smem)) != MD_OK) return s;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min(num_sms(), pl.units));
+  cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3((kConsumerWarps + 1) * 32);
   cfg.dynamicSmemBytes = v_smem;
   cfg.stream = st;
@@ -139,7 +139,8 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   MergeArgs ma;
   ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
-  ma.K = pl.K; ma.kmax = pl.kmax; ma.ntiles = pl.ntiles;
+  ma.K = pl.K; ma.kmax = pl.kmax; ma.nslots = pl.grid;
+  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
   heads_merge_kernel<<<pl.M * pl.K, 256, 0, st>>>(ma);
   return last_launch();
@@ -233,7 +234,8 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   md::heads::MergeArgs ma;
   ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
-  ma.K = K; ma.kmax = kmax; ma.ntiles = pl.ntiles2;
+  ma.K = K; ma.kmax = kmax; ma.nslots = pl.ntiles2;
+  ma.partitioned = 0; ma.units = 0; ma.ntiles = pl.ntiles2;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
   md::heads::heads_merge_kernel<<<M * K, 256, 0, st>>>(ma);
   return last_launch();
@@ -275,7 +277,7 @@ struct AttnPlan {
   bool tc;                  // tensor-core path (the GQA group divides 128)
   int G, R, max_chunks;     // CUDA-core path
   int rtiles, splits, cps;  // tensor-core path
-  size_t off_ml, bytes;
+  size_t off_ml, off_cnt, bytes;
 };
 
 AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
@@ -285,23 +287,25 @@ AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
   p.R = T * p.G;
   p.tc = (128 % p.G) == 0;
   if (p.tc) {
+    // one wave of CTAs: (splits x row tiles x KV heads x requests) <= #SMs
     p.rtiles = (p.R + 127) / 128;
     const int chunks = (S_max + md::attn_tc::kBN - 1) / md::attn_tc::kBN;
     const int base = B * Hkv * p.rtiles;
-    int splits = (num_sms() + base - 1) / base;
-    splits = std::max(1, std::min(splits, chunks));
+    int splits = std::max(1, num_sms() / base);
+    splits = std::min(std::min(splits, chunks), md::attn_tc::kMaxSplits);
     p.cps = (chunks + splits - 1) / splits;
     p.splits = (chunks + p.cps - 1) / p.cps;
     p.max_chunks = chunks;
-    const size_t rows = size_t(B) * Hkv * p.splits * p.rtiles * 128;
+    const size_t rows = size_t(base) * p.splits * 128;
     p.off_ml = align256(rows * dh * 4);
-    p.bytes = p.off_ml + align256(rows * 8);
+    p.off_cnt = p.off_ml + align256(rows * 8);
+    p.bytes = p.off_cnt + align256(size_t(base) * 4);
   } else {
     p.rtiles = p.splits = p.cps = 0;
     p.max_chunks = (S_max + md::attn::kChunk - 1) / md::attn::kChunk;
     const size_t rows = size_t(B) * Hkv * p.max_chunks * p.R;
     p.off_ml = align256(rows * dh * 4);
-    p.bytes = p.off_ml + align256(rows * 8);
+    p.off_cnt = p.bytes = p.off_ml + align256(rows * 8);
   }
   return p;
 }
@@ -333,15 +337,15 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   a.prefix_len = prefix_len;
   a.part_o = static_cast<float*>(ws);
   a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
+  a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pl.off_cnt);
   a.out = out;
   a.B = B; a.S_max = S_max; a.Hq = Hq; a.Hkv = Hkv; a.G = pl.G; a.R = pl.R; a.rtiles = pl.rtiles;
   a.splits = pl.splits; a.chunks_per_split = pl.cps;
   a.scale_log2 = sc * 1.4426950408889634f;
+  if ((s = cuda_ok(cudaMemsetAsync(a.counters, 0, size_t(B) * Hkv * pl.rtiles * 4, st))) != MD_OK) return s;
   constexpr int sm = Cfg<DH>::kSmem;
   if ((s = set_smem(attn_tc_kernel<DH>, sm)) != MD_OK) return s;
   attn_tc_kernel<DH><<<dim3(pl.splits, Hkv * pl.rtiles, B), kThreads, sm, st>>>(qmap, kmap, vmap, tree->tp, a);
-  if ((s = last_launch()) != MD_OK) return s;
-  attn_tc_merge_kernel<DH><<<dim3(T * Hq, B), DH, 0, st>>>(tree->tp, a);
   return last_launch();
 }
 

@@ -72,7 +72,11 @@ LLAMA70B_CHAIN = replace(LLAMA70B, name="llama3-70b-chain", k_per_head=(1, 1, 1,
                          accept=CHAIN_ACCEPT)
 BATCHED70B = replace(LLAMA70B, name="llama3-70b-b8", B=8, prefix=(1024, 8192), heads_rows="BT")
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B)}
+# Profiling case for the heads kernels: 8B-shaped with a 32000-token vocabulary,
+# so the weights (1.1 GB) exceed L2 while the device footprint stays small.
+PROF_HEADS = replace(LLAMA8B, name="prof-8b-v32000", V=32000)
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS)}
 
 
 def sweep_8b(B: int, tree: str, prefix: int, mode: str = "greedy") -> Workload:
