@@ -51,6 +51,26 @@ def heads_bytes(w):
     return weights + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax
 
 
+def slowest_rank_ms(ms: float, world: int, device=None) -> float:
+    """Elapsed milliseconds of the slowest rank (all-reduce MAX; a no-op on one rank)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job steps/s: every rank ran `steps` steps within the slowest rank's time."""
+    return world * steps / (max_ms / 1000.0)
+
+
+def heads_flops(w):
+    return 2 * w.M * w.K * w.d * (w.d + w.V)
+
+
 def attention_bytes(w, P):
     kv = sum(2 * w.Hkv * (int(p) + w.T) * w.dh * 2 for p in P)
     return kv + w.B * w.T * w.Hq * w.dh * (2 + 4)
@@ -290,14 +310,14 @@ def run_medusa(args, w):
     stream.synchronize()
     tokens = step.tokens.cpu().numpy()
     parent_np = np.array(step.tree.parent)
-    logits_host = synth.planted_logits(seed, parent_np, tokens, w.V, w.accept, sigma=w.logit_sigma, bump=w.bump)
+    logits_dev = synth.planted_logits_device(seed, parent_np, tokens, w.V, w.accept, sigma=w.logit_sigma,
+                                             bump=w.bump, device=dev)
     sets = []
     for i in range(nsets):
         q = sdev.fill_normal(torch.empty((w.B, w.T, w.Hq, w.dh), **bf), seed + 7919 * i, "q", 1.0)
         kc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + 7919 * i, "k_cache", 1.0)
         vc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + 7919 * i, "v_cache", 1.0)
-        lg = torch.from_numpy(logits_host).to(dev)
-        sets.append((q, kc, vc, lg))
+        sets.append((q, kc, vc, logits_dev.clone()))
     torch.cuda.synchronize()
 
     def one_step(i, ev=None):
@@ -346,12 +366,9 @@ def run_medusa(args, w):
     per_call = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
     clk = clocks.summary()
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = slowest_rank_ms(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * args.steps / (total_ms / 1000.0)
+    value = job_value(world, args.steps, total_ms)
 
     # ---- end to end through the public API with host buffers ---------------
     e2e = None
@@ -361,8 +378,21 @@ def run_medusa(args, w):
     if rank == 0:
         peaks = measured_peaks()
         hb = heads_bytes(w)
+        hf = heads_flops(w)
         heads_ms = float(per_call[:, 0].mean())
-        achieved = hb / (heads_ms / 1000.0) / 1e9
+        if w.M > 8:      # tensor-core GEMM path: bound by the bf16 tensor pipe
+            roof = {"kernel": "md_medusa_heads (tcgen05 GEMMs: residual block, vocabulary projection + top-k; merge)",
+                    "bound": "tensor", "achieved": hf / (heads_ms / 1000.0) / 1e12,
+                    "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "algorithmic_flops": hf, "peak_note": "measured cuBLAS bf16, sustained (kernel inside a long step)"}
+        else:
+            roof = {"kernel": "md_medusa_heads (residual block + vocabulary stream + top-k merge)",
+                    "bound": "hbm", "achieved": hb / (heads_ms / 1000.0) / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "algorithmic_bytes": hb, "peak_note": "measured copy bandwidth"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = args.traffic
+        roof["avg_ms"] = heads_ms
+        roof["peak_source"] = peaks["source"]
         ab = attention_bytes(w, P)
         af = attention_flops(w, P)
         attn_ms = float(per_call[:, 2].mean())
@@ -375,10 +405,7 @@ def run_medusa(args, w):
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, P),
-            "roofline": {"kernel": "md_medusa_heads (residual block + vocabulary stream + top-k merge)",
-                         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": args.traffic,
-                         "algorithmic_bytes": hb, "avg_ms": heads_ms, "peak_source": peaks["source"]},
+            "roofline": roof,
             "step_gbs": step_bytes / (ms_per_step / 1000.0) / 1e9 / 1.0,
             "step_gbs_frac": step_bytes / (ms_per_step / 1000.0) / 1e9 / peaks["hbm_gbs"],
             "per_call_ms": {"medusa_heads": heads_ms, "tree_build": float(per_call[:, 1].mean()),
@@ -463,6 +490,77 @@ def run_part(args, w):
                       "device_status": status}), flush=True)
 
 
+def run_sweep(args):
+    """The 8B-shaped sweep: B x tree x KV prefix x acceptance rule, one JSON line
+    per point with the per-call times (device, CUDA events, eager)."""
+    import torch
+
+    import medusa_draft_heads_b200 as md
+    from medusa_draft_heads_b200.step import MedusaStep
+    from seeded_inputs import device as sdev
+    from seeded_inputs.workloads import sweep_8b
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    base = sweep_8b(1, "64", 1024)
+    W1 = sdev.fill_normal(torch.empty((base.K, base.d, base.d), **bf), base.seed, "W1", base.w_sigma)
+    b1 = sdev.fill_normal(torch.empty((base.K, base.d), **bf), base.seed, "b1", base.w_sigma)
+    Wv = sdev.fill_normal(torch.empty((base.K, base.d, base.V), **bf), base.seed, "Wv", base.w_sigma)
+    Bs = [int(x) for x in args.sweep_batches.split(",")]
+    for mode in args.sweep_modes.split(","):
+        for tree in ("chain", "16", "64"):
+            for P in (1024, 8192, 32768):
+                for B in Bs:
+                    w = sweep_8b(B, tree, P, mode)
+                    tups = md.select_tree(w.k_per_head, w.accept, w.n_nodes)
+                    step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups,
+                                      Hq=w.Hq, Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode,
+                                      temperature=w.temperature, eps=w.eps, alpha=w.alpha, device=dev)
+                    h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), w.seed + B, "h", 1.0)
+                    root = torch.from_numpy(synth.root_tokens(w.seed + B, w.B, w.V)).to(dev)
+                    prefix = torch.full((w.B,), P, dtype=torch.int32, device=dev)
+                    q = sdev.fill_normal(torch.empty((w.B, w.T, w.Hq, w.dh), **bf), w.seed + B, "q", 1.0)
+                    kc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), w.seed + B, "k_cache", 1.0)
+                    vc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), w.seed + B, "v_cache", 1.0)
+                    with torch.cuda.stream(stream):
+                        step.heads(h, W1, b1, Wv)
+                        step.build(root, prefix)
+                    stream.synchronize()
+                    lg = synth.planted_logits_device(w.seed + B, np.array(step.tree.parent), step.tokens.cpu().numpy(),
+                                                     w.V, w.accept, sigma=w.logit_sigma, bump=w.bump, device=dev)
+                    torch.cuda.synchronize()
+                    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+                    with torch.cuda.stream(stream):
+                        for i in range(args.warmup + args.steps):
+                            ev = evs[i - args.warmup] if i >= args.warmup else None
+                            if ev: ev[0].record(stream)
+                            step.heads(h, W1, b1, Wv)
+                            if ev: ev[1].record(stream)
+                            step.build(root, prefix)
+                            if ev: ev[2].record(stream)
+                            step.attention(q, kc, vc, prefix)
+                            if ev: ev[3].record(stream)
+                            step.accept(lg)
+                            if ev: ev[4].record(stream)
+                    torch.cuda.synchronize()
+                    status = md.device_status(stream=stream)
+                    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+                    tot = float(np.mean([e[0].elapsed_time(e[4]) for e in evs]))
+                    print(json.dumps({"sweep": w.name, "B": B, "tree": tree, "prefix": P, "mode": mode,
+                                      "heads_path": "tcgen05-gemm" if w.M > 8 else "cuda-core-stream",
+                                      "steps_per_s": 1000.0 / tot, "ms_per_step": tot,
+                                      "ms": {"heads": float(per[:, 0].mean()), "build": float(per[:, 1].mean()),
+                                             "attention": float(per[:, 2].mean()),
+                                             "accept": float(per[:, 3].mean())},
+                                      "attention_tflops": attention_flops(w, [P] * B) / (per[:, 2].mean() / 1e3) / 1e12,
+                                      "accept_len_mean": float(step.accept_len.float().mean().item()),
+                                      "device_status": status}), flush=True)
+                    del step, h, q, kc, vc, lg
+                    torch.cuda.empty_cache()
+
+
 def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, dev, world, barrier):
     """Same step through the public API, with this step's inputs copied from
     pinned host memory and the result read back every step."""
@@ -509,13 +607,8 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
         e.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = s.elapsed_time(e)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": world * steps / (ms / 1000.0), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+    ms = slowest_rank_ms(s.elapsed_time(e), world, dev)
+    return {"value": job_value(world, steps, ms), "unit": "steps/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "per step: h, root token, prefix lengths, q, the tree tokens' K/V and the target logits "
                     "copied in from pinned host memory; accept_len, path and bonus copied out; stream "
@@ -546,6 +639,10 @@ def main():
     ap.add_argument("--workload", default="llama3-70b", choices=sorted(WORKLOADS))
     ap.add_argument("--part", choices=["step", "heads", "attention", "accept"], default="step",
                     help="time one call alone (profiling); the JSON line then reports that call only")
+    ap.add_argument("--sweep", action="store_true",
+                    help="run the 8B-shaped sweep (B x tree x prefix x rule), one JSON line per point")
+    ap.add_argument("--sweep-batches", default="1,2,4,8,16,32")
+    ap.add_argument("--sweep-modes", default="greedy,typical")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-frac", type=float, default=1 / 64)
@@ -557,6 +654,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.part != "step":
         run_part(args, w)
         return

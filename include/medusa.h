@@ -71,8 +71,8 @@ enum {
 
 /* Supported ranges (anything else: MD_ERR_UNSUPPORTED).
  *   heads:     1 <= K <= 8, 1 <= k_i <= kmax <= 16, d % 64 == 0, V % 8 == 0,
- *              V >= 256, 1 <= M <= 4096 (M <= 8: CUDA-core weight stream;
- *              M > 8: tcgen05 tensor-core GEMM, h and b1 16-byte aligned).
+ *              V >= 256, 1 <= M <= 4096 (M <= 4: CUDA-core weight stream;
+ *              M > 4: tcgen05 tensor-core GEMM, h and b1 16-byte aligned).
  *   tree:      1 <= T <= 128, depth <= K.
  *   attention: dh in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16.
  */
@@ -162,8 +162,7 @@ MD_API md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_b
  *
  * - Sizes whose scratch (md_heads_workspace) exceeds the array are rejected
  *   with MD_ERR_WORKSPACE before anything is launched (at d = 8192,
- *   V = 128256, K = 4, kmax = 10 this admits M <= 6, and M = 9 .. 37 on the
- *   tensor-core path).
+ *   V = 128256, K = 4, kmax = 10 this admits M <= 74).
  * - The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
  *   first call before any stream capture on the device.

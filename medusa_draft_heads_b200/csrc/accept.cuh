@@ -70,6 +70,8 @@ __device__ __forceinline__ void soft_add(Soft& s, float y) {
 }
 
 __global__ void __launch_bounds__(kRowThreads) accept_rows_kernel(Args a) {
+  pdl_wait_primary();          // logits and tokens may come from earlier kernels
+  pdl_launch_dependents();
   const int row = blockIdx.y, c = blockIdx.x;
   const int v0 = c * a.chunk_len;
   const int v1 = min(a.V, v0 + a.chunk_len);
@@ -149,6 +151,8 @@ __global__ void __launch_bounds__(kRowThreads) accept_rows_kernel(Args a) {
 }
 
 __global__ void __launch_bounds__(MD_MAX_T) accept_walk_kernel(const __grid_constant__ TreeParams tp, Args a) {
+  pdl_wait_primary();          // row summaries come from accept_rows_kernel
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   const int j = threadIdx.x;
   const int T = tp.T;

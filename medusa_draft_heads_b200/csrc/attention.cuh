@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(kThreads) attn_chunk_kernel(const __grid_const
   float* qs = reinterpret_cast<float*>(Vs + kChunk * DH);
   const int c = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int T = tp.T;
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int P = a.prefix_len[b];
   if (P < 0 || P + T > a.S_max) {
     if (c == 0 && hk == 0 && threadIdx.x == 0) set_status(MD_DEV_BAD_PREFIX);
@@ -155,6 +157,8 @@ __global__ void __launch_bounds__(kThreads) attn_chunk_kernel(const __grid_const
 // grid (T * Hq, B), DH threads (one output dimension each).
 template <int DH>
 __global__ void __launch_bounds__(DH) attn_merge_kernel(const __grid_constant__ TreeParams tp, Args a) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int b = blockIdx.y;
   const int th = blockIdx.x;
   const int t = th / a.Hq, h = th % a.Hq;

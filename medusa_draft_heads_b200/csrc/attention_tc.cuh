@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int split = blockIdx.x, rt = blockIdx.y % a.rtiles, hk = blockIdx.y / a.rtiles, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = tp.T;
+  pdl_wait_primary();          // inputs may come from earlier kernels
+  pdl_launch_dependents();
   const int P = a.prefix_len[b];
   const bool bad = P < 0 || P + T > a.S_max;
   const int nkeys = bad ? 0 : P + T;

@@ -27,7 +27,7 @@ constexpr int kZPad = 8;            // z row i is stored as 8 bf16 (one per m), 
 constexpr int kW1Threads = 256;
 constexpr int kW1TileO = 256;       // phase-1 output columns per CTA
 constexpr int kW1MaxRows = 1024;    // phase-1 hidden rows per CTA (split-K)
-constexpr int kMaxM = 8;
+constexpr int kMaxM = 4;        // rows beyond this take the tensor-core path (faster from M = 5 on)
 constexpr uint32_t kStageWBytes = kStageRows * kTileV * 2;  // 32 KB
 constexpr uint32_t kStageZBytes = kStageRows * kZPad * 2;   // 1 KB
 constexpr int kSmemBudget = 227 * 1024;
@@ -251,6 +251,7 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int stages_per_unit = a.d / kStageRows;
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
@@ -443,8 +444,10 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 // ---------------------------------------------------------------------------
 // Phase 3: merge candidate lists into each head's top-k.
 // grid (M * K), 256 threads. The candidates of (m, k) are `nslots` lists of
-// up to kmax entries. In "partitioned" mode slot c is CTA c of the vocabulary
-// kernel and only CTAs whose unit range touches head k wrote a list. Each
+// up to kmax entries. In "partitioned" mode slot c is CTA c of the kernel that
+// produced them: that kernel split `units` work units, ordered (row tile of
+// `mrows` rows, head, column tile of `ntiles`), into contiguous CTA ranges, and
+// only CTAs whose range touches the (row tile of m, head k) run wrote a list. Each
 // thread gathers its slots into a sorted register list; each warp then merges
 // its 32 lists by k rounds of a shuffle arg-max over the list heads (the
 // winning lane shifts its list), and warp 0 merges the 8 warp lists the same way.
@@ -455,7 +458,7 @@ struct MergeArgs {
   int32_t* topk_ids;   // [M, K, kmax]
   float* topk_vals;
   int K, kmax, nslots;
-  int partitioned, units, ntiles;   // vocabulary-kernel partition (partitioned == 1)
+  int partitioned, units, ntiles, mrows;   // producer partition (partitioned == 1)
   int kph[MD_MAX_K];
 };
 
@@ -519,19 +522,22 @@ __device__ __forceinline__ void warp_merge(SortedList& L, int kk, int lane, floa
 }
 
 __global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
+  pdl_wait_primary();          // candidates come from the previous kernel
+  pdl_launch_dependents();
   __shared__ float wv[8][kListMax];
   __shared__ int wi[8][kListMax];
   const int mk = blockIdx.x;
-  const int k = mk % a.K;
+  const int k = mk % a.K, m = mk / a.K;
   const int kk = a.kph[k];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t base = size_t(mk) * a.nslots * a.kmax;
+  const long long run = (long long)(m / a.mrows) * a.K + k;   // (row tile, head) run of (m, k)
   SortedList L;
   L.clear();
   for (int c = threadIdx.x; c < a.nslots; c += 256) {
     if (a.partitioned) {
       const long long u0 = (long long)c * a.units / a.nslots, u1 = (long long)(c + 1) * a.units / a.nslots;
-      if (u1 <= (long long)k * a.ntiles || u0 >= (long long)(k + 1) * a.ntiles) continue;
+      if (u1 <= run * a.ntiles || u0 >= (run + 1) * a.ntiles) continue;
     }
     for (int j = 0; j < kk; ++j) {
       const int id = a.cand_id[base + size_t(c) * a.kmax + j];

@@ -17,6 +17,13 @@
 // TMA, one thread of warp 1 issues tcgen05.mma into one of two 128 x 256 fp32
 // accumulators in tensor memory (512 columns), warps 2..5 drain the other
 // accumulator through tcgen05.ld (one TMEM lane = one row per thread).
+//
+// Tiles are ordered (row tile, head, column tile) and CTA c takes the
+// contiguous range [c*U/G, (c+1)*U/G), so the CTAs working on different row
+// tiles walk the same weight columns at the same time (the weight strip is
+// read from HBM once and then from L2), and in phase 2 each row keeps one
+// running top-k across the CTA's column tiles: after the first tiles nearly
+// every logit is rejected by one compare against the current k-th best.
 #pragma once
 
 #include "common.cuh"
@@ -31,7 +38,7 @@ constexpr uint32_t kBBox = kBK * 64 * 2;        // 8 KB: 64 k-rows x 64 n-column
 constexpr uint32_t kBBytes = 4 * kBBox;         // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 192;
-constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
+constexpr int kSmem = kStages * kStageBytes + 1024 + 256 + MD_MAX_KMAX * 128 * 8;   // + running lists
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxM = 4096;
 
@@ -39,44 +46,45 @@ enum { EPI_SILU = 0, EPI_TOPK = 1 };
 
 struct Args {
   int M, d, N, K;                 // rows, reduction length, output columns, heads
-  int mtiles, ntiles, tiles;
+  int mtiles, ntiles, tiles;      // tiles = mtiles * K * ntiles, ordered (mtile, head, ntile)
   int a_shared;                   // A is one matrix for every head (phase 1: h)
   const uint16_t* h;              // [M, d]      phase 1 residual
   const uint16_t* b1;             // [K, d]      phase 1 bias
   uint16_t* zg;                   // [K, M, d]   phase 1 output
-  float* cand_val;                // [M, K, ntiles, kmax]  phase 2 output
+  float* cand_val;                // [M, K, gridDim.x, kmax]  phase 2: one list per (row, head, CTA)
   int* cand_id;
   float* logits_dbg;              // [M, K, N] or null
   int kmax;
   int kph[MD_MAX_K];
 };
 
-template <int KK>
-struct TopK {
-  float v[KK];
-  int i[KK];
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int j = 0; j < KK; ++j) {
-      v[j] = -INFINITY;
-      i[j] = INT_MAX;
+// Running top-k of one row in shared memory: entry j of thread t at
+// [j * 128 + t] (conflict-free across a warp); sorted, best first.
+struct SmemList {
+  float* v;
+  int* i;
+  int kk;
+  float tv;   // the current k-th best (the admission threshold)
+  int ti;
+  __device__ __forceinline__ void reset() {
+    for (int j = 0; j < kk; ++j) {
+      v[j * 128] = -INFINITY;
+      i[j * 128] = INT_MAX;
     }
+    tv = -INFINITY;
+    ti = INT_MAX;
   }
-  __device__ __forceinline__ void push(float x, int id) {
-    if (!better(x, id, v[KK - 1], i[KK - 1])) return;
-    v[KK - 1] = x;
-    i[KK - 1] = id;
-#pragma unroll
-    for (int j = KK - 1; j > 0; --j) {
-      if (better(v[j], i[j], v[j - 1], i[j - 1])) {
-        const float tv = v[j];
-        v[j] = v[j - 1];
-        v[j - 1] = tv;
-        const int ti = i[j];
-        i[j] = i[j - 1];
-        i[j - 1] = ti;
-      }
+  __device__ __forceinline__ void insert(float x, int id) {
+    int pos = kk - 1;
+    while (pos > 0 && better(x, id, v[(pos - 1) * 128], i[(pos - 1) * 128])) {
+      v[pos * 128] = v[(pos - 1) * 128];
+      i[pos * 128] = i[(pos - 1) * 128];
+      --pos;
     }
+    v[pos * 128] = x;
+    i[pos * 128] = id;
+    tv = v[(kk - 1) * 128];
+    ti = i[(kk - 1) * 128];
   }
 };
 
@@ -90,9 +98,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  float* lv = reinterpret_cast<float*>(smem + kStages * kStageBytes + 256);    // [kmax][128] running lists
+  int* li = reinterpret_cast<int*>(lv + MD_MAX_KMAX * 128);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = a.d / kBK;
+  const int t_begin = int((long long)blockIdx.x * a.tiles / gridDim.x);
+  const int t_end = int((long long)(blockIdx.x + 1) * a.tiles / gridDim.x);
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -123,9 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol = policy_evict_first();
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
-        const int mt = tile % a.mtiles, r = tile / a.mtiles;
-        const int nt = r % a.ntiles, k = r / a.ntiles;
+      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        const int nt = tile % a.ntiles, r = tile / a.ntiles;
+        const int k = r % a.K, mt = r / a.K;
         for (int s = 0; s < nk; ++s, ++it) {
           const int slot = it % kStages;
           if (it >= kStages && !mbar_wait(smem_u32(&empty[slot]), ((it / kStages) - 1) & 1)) {
@@ -155,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = umma_idesc_bf16(kBM, kBN, 0, 1);
       int it = 0, lt = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++lt) {
+      for (int tile = t_begin; tile < t_end && ok; ++tile, ++lt) {
         const int buf = lt & 1;
         if (lt >= 2 && !mbar_wait(smem_u32(&acc_empty[buf]), ((lt >> 1) - 1) & 1)) {
           set_status(MD_DEV_TIMEOUT);
@@ -187,10 +200,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------- epilogue ----------------------------------
     const int q = warp & 3;   // TMEM lanes 32q .. 32q+31 belong to this warp
     const int row = q * 32 + lane;
+    SmemList L;
+    L.v = lv + row;
+    L.i = li + row;
     int lt = 0;
-    for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++lt) {
-      const int mt = tile % a.mtiles, r = tile / a.mtiles;
-      const int nt = r % a.ntiles, k = r / a.ntiles;
+    int cur_k = -1;
+    for (int tile = t_begin; tile < t_end; ++tile, ++lt) {
+      const int nt = tile % a.ntiles, r = tile / a.ntiles;
+      const int k = r % a.K, mt = r / a.K;
       const int buf = lt & 1;
       if (!mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1)) {
         set_status(MD_DEV_TIMEOUT);
@@ -228,8 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        TopK<KK> tk;
-        tk.init();
+        if (k != cur_k) {         // a new (row tile, head) run starts: fresh lists
+          L.kk = a.kph[k];
+          L.reset();
+          cur_k = k;
+        }
         for (int c = 0; c < kBN; c += 32) {
           float v[32];
           tmem_ld32(tbase + c, v);
@@ -237,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (live) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (c0 + j < a.N) tk.push(v[j], c0 + j);
+              if (c0 + j < a.N && better(v[j], c0 + j, L.tv, L.ti)) L.insert(v[j], c0 + j);
             if (a.logits_dbg) {
               float* lp = a.logits_dbg + (size_t(m) * a.K + k) * a.N + c0;
 #pragma unroll
@@ -246,16 +266,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (live) {
-          const int kk = a.kph[k];
-          const size_t cb = ((size_t(m) * a.K + k) * a.ntiles + nt) * a.kmax;
-#pragma unroll
-          for (int j = 0; j < KK; ++j) {
-            if (j < kk) {
-              a.cand_val[cb + j] = tk.v[j];
-              a.cand_id[cb + j] = tk.i[j] == INT_MAX ? -1 : tk.i[j];
+        // flush at the end of a (row tile, head) run
+        const bool last = tile + 1 == t_end || (tile + 1) / a.ntiles != tile / a.ntiles;
+        if (last) {
+          if (live) {
+            const size_t cb = ((size_t(m) * a.K + k) * gridDim.x + blockIdx.x) * a.kmax;
+            for (int j = 0; j < L.kk; ++j) {
+              a.cand_val[cb + j] = L.v[j * 128];
+              a.cand_id[cb + j] = L.i[j * 128] == INT_MAX ? -1 : L.i[j * 128];
             }
           }
+          cur_k = -1;
         }
       }
       tc_fence_before();

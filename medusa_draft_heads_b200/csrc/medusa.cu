@@ -6,6 +6,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 
 #include "common.cuh"
 #include "heads.cuh"
@@ -84,6 +85,25 @@ md_status make_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_
   return r == CUDA_SUCCESS ? MD_OK : MD_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while its predecessor on the stream finishes; it waits (griddepcontrol.wait)
+// before reading anything the predecessor writes.
+template <typename... KArgs, typename... Args>
+md_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
+
 template <typename Kernel>
 md_status set_smem(Kernel k, int bytes) {
   return cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
@@ -140,16 +160,16 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = pl.K; ma.kmax = pl.kmax; ma.nslots = pl.grid;
-  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles;
+  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.mrows = 1 << 30;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
-  heads_merge_kernel<<<pl.M * pl.K, 256, 0, st>>>(ma);
-  return last_launch();
+  return launch_pdl(heads_merge_kernel, dim3(pl.M * pl.K), dim3(256), 0, st, ma);
 }
 
 // Workspace of the tensor-core path (M > 8): z [K, M, d] bf16 and the
 // per-tile candidates [M, K, ceil(V/256), kmax].
 struct GemmPlan {
   int mtiles, ntiles1, ntiles2;
+  int grid1, grid2;   // CTAs of the two GEMMs (one candidate list per row, head and CTA in phase 2)
   size_t off_z, off_cval, off_cid, bytes;
 };
 
@@ -159,10 +179,12 @@ GemmPlan gemm_plan(int M, int d, int V, int K, int kmax) {
   p.mtiles = (M + md::gemm::kBM - 1) / md::gemm::kBM;
   p.ntiles1 = (d + md::gemm::kBN - 1) / md::gemm::kBN;
   p.ntiles2 = (V + md::gemm::kBN - 1) / md::gemm::kBN;
+  p.grid1 = std::min(num_sms(), K * p.ntiles1 * p.mtiles);
+  p.grid2 = std::min(num_sms(), K * p.ntiles2 * p.mtiles);
   size_t o = 0;
   p.off_z = o;    o = align256(o + size_t(K) * M * d * 2);
-  p.off_cval = o; o = align256(o + size_t(M) * K * p.ntiles2 * kmax * 4);
-  p.off_cid = o;  o = align256(o + size_t(M) * K * p.ntiles2 * kmax * 4);
+  p.off_cval = o; o = align256(o + size_t(M) * K * p.grid2 * kmax * 4);
+  p.off_cid = o;  o = align256(o + size_t(M) * K * p.grid2 * kmax * 4);
   p.bytes = o;
   return p;
 }
@@ -234,11 +256,10 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   md::heads::MergeArgs ma;
   ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
-  ma.K = K; ma.kmax = kmax; ma.nslots = pl.ntiles2;
-  ma.partitioned = 0; ma.units = 0; ma.ntiles = pl.ntiles2;
+  ma.K = K; ma.kmax = kmax; ma.nslots = pl.grid2;
+  ma.partitioned = 1; ma.units = K * pl.ntiles2 * pl.mtiles; ma.ntiles = pl.ntiles2; ma.mrows = kBM;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
-  md::heads::heads_merge_kernel<<<M * K, 256, 0, st>>>(ma);
-  return last_launch();
+  return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
 }
 
 md_status heads_check(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax) {
@@ -345,6 +366,7 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   if ((s = cuda_ok(cudaMemsetAsync(a.counters, 0, size_t(B) * Hkv * pl.rtiles * 4, st))) != MD_OK) return s;
   constexpr int sm = Cfg<DH>::kSmem;
   if ((s = set_smem(attn_tc_kernel<DH>, sm)) != MD_OK) return s;
+  // ordinary launch: the counters were just zeroed by a memset on this stream
   attn_tc_kernel<DH><<<dim3(pl.splits, Hkv * pl.rtiles, B), kThreads, sm, st>>>(qmap, kmap, vmap, tree->tp, a);
   return last_launch();
 }
@@ -476,10 +498,6 @@ md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1
     case 2: return launch_heads<2>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
     case 3: return launch_heads<3>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
     case 4: return launch_heads<4>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 5: return launch_heads<5>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 6: return launch_heads<6>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 7: return launch_heads<7>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 8: return launch_heads<8>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
     default: return MD_ERR_UNSUPPORTED;
   }
 }
@@ -510,8 +528,8 @@ md_status md_tree_build(const md_tree* tree, const int32_t* topk_ids, int32_t M,
   a.topk_ids = topk_ids; a.head_row = head_row; a.root_token = root_token; a.prefix_len = prefix_len;
   a.tokens = tokens; a.parent = parent; a.anc = anc; a.pos = pos;
   a.M = M; a.K = tree->K; a.kmax = kmax;
-  md::tree::tree_build_kernel<<<B, MD_MAX_T, 0, static_cast<cudaStream_t>(stream)>>>(tree->tp, a);
-  return last_launch();
+  return launch_pdl(md::tree::tree_build_kernel, dim3(B), dim3(MD_MAX_T), 0, static_cast<cudaStream_t>(stream),
+                    tree->tp, a);
 }
 
 md_status md_attention_workspace(int32_t B, int32_t T, int32_t Hq, int32_t Hkv, int32_t dh, int32_t S_max,
@@ -597,10 +615,10 @@ md_status md_tree_accept(const float* logits, int32_t V, const int32_t* tokens, 
   a.log_eps = std::log(eps);
   a.log_alpha = std::log(alpha);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  md::acc::accept_rows_kernel<<<dim3(pl.nchunks, B * T), md::acc::kRowThreads, 0, st>>>(a);
-  if ((s = last_launch()) != MD_OK) return s;
-  md::acc::accept_walk_kernel<<<B, MD_MAX_T, 0, st>>>(tree->tp, a);
-  return last_launch();
+  if ((s = launch_pdl(md::acc::accept_rows_kernel, dim3(pl.nchunks, B * T), dim3(md::acc::kRowThreads), 0, st, a)) !=
+      MD_OK)
+    return s;
+  return launch_pdl(md::acc::accept_walk_kernel, dim3(B), dim3(MD_MAX_T), 0, st, tree->tp, a);
 }
 
 md_status md_get_device_status(void* stream, int32_t* out, int32_t clear) {

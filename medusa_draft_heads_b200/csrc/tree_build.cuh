@@ -24,6 +24,8 @@ struct BuildArgs {
 };
 
 __global__ void __launch_bounds__(MD_MAX_T) tree_build_kernel(const __grid_constant__ TreeParams tp, BuildArgs a) {
+  pdl_wait_primary();          // top-k ids come from the previous kernel
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   const int j = threadIdx.x;
   __shared__ int row_ok;

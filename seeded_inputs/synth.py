@@ -67,6 +67,35 @@ def synthetic_tree_tokens(seed: int, B: int, parent, V: int, root_tokens=None) -
     return out.astype(np.int32)
 
 
+def plant_choices(seed: int, parent, tokens, V: int, accept):
+    """The planting decisions: (b, p, x) = raise token x of row (b, p)."""
+    tokens = np.asarray(tokens)
+    B, T = tokens.shape
+    depth = node_depths(parent)
+    ch = children_lists(parent)
+    kp = stream_key(seed, "plant")
+    kq = stream_key(seed, "plant_pick")
+    out = []
+    for b in range(B):
+        for p in range(T):
+            if not ch[p]:
+                continue
+            idx = np.array([b * T + p])
+            u = float(uniform_unit_at(kp, idx)[0])
+            child_tokens = sorted({int(tokens[b, c]) for c in ch[p]})
+            if u < accept[int(depth[p])]:
+                c = ch[p][int(uniform_int_at(kq, idx, len(ch[p]))[0])]
+                x = int(tokens[b, c])
+            else:
+                j = int(uniform_int_at(kq, idx, V - len(child_tokens))[0])
+                for t in child_tokens:  # j-th token id that is not a child token
+                    if t <= j:
+                        j += 1
+                x = j
+            out.append((b, p, x))
+    return out
+
+
 def planted_logits(seed: int, parent, tokens, V: int, accept, sigma: float = 1.0,
                    bump: float = 1.0, logits: np.ndarray | None = None) -> np.ndarray:
     """Target logits fp32 [B, T, V] with the acceptance profile planted.
@@ -78,30 +107,31 @@ def planted_logits(seed: int, parent, tokens, V: int, accept, sigma: float = 1.0
     B, T = tokens.shape
     if logits is None:
         logits = normal_f32(seed, "logits", (B, T, V), sigma)
-    depth = node_depths(parent)
-    ch = children_lists(parent)
-    kp = stream_key(seed, "plant")
-    kq = stream_key(seed, "plant_pick")
     bump32 = np.float32(bump)
-    for b in range(B):
-        for p in range(T):
-            if not ch[p]:
-                continue
-            idx = np.array([b * T + p])
-            u = float(uniform_unit_at(kp, idx)[0])
-            row = logits[b, p]
-            top = np.float32(row.max())
-            child_tokens = sorted({int(tokens[b, c]) for c in ch[p]})
-            if u < accept[int(depth[p])]:
-                c = ch[p][int(uniform_int_at(kq, idx, len(ch[p]))[0])]
-                x = int(tokens[b, c])
-            else:
-                j = int(uniform_int_at(kq, idx, V - len(child_tokens))[0])
-                for t in child_tokens:  # j-th token id that is not a child token
-                    if t <= j:
-                        j += 1
-                x = j
-            row[x] = np.float32(top + bump32)
+    for b, p, x in plant_choices(seed, parent, tokens, V, accept):
+        row = logits[b, p]
+        row[x] = np.float32(np.float32(row.max()) + bump32)
+    return logits
+
+
+def planted_logits_device(seed: int, parent, tokens, V: int, accept, sigma: float = 1.0,
+                          bump: float = 1.0, device="cuda"):
+    """The same tensor as planted_logits, drawn and planted on the GPU (torch
+    float32 tensor): the draws come from the device twin of the generator and
+    each planted value is the same fp32 sum row max + bump."""
+    import torch
+
+    from .device import fill_normal
+    tokens = np.asarray(tokens)
+    B, T = tokens.shape
+    logits = fill_normal(torch.empty((B, T, V), dtype=torch.float32, device=device), seed, "logits", sigma)
+    ch = plant_choices(seed, parent, tokens, V, accept)
+    if ch:
+        b = torch.tensor([c[0] for c in ch], device=device)
+        p = torch.tensor([c[1] for c in ch], device=device)
+        x = torch.tensor([c[2] for c in ch], device=device)
+        top = logits[b, p].amax(dim=-1)
+        logits[b, p, x] = top + torch.tensor(bump, dtype=torch.float32, device=device)
     return logits
 
 

@@ -63,8 +63,8 @@ def test_static_scratch_matches_workspace_call(M, d, V, kph):
 
 
 def test_static_scratch_refuses_oversized_shapes():
-    """M = 8 rows of 70B-shaped heads need more scratch than the array holds."""
-    M, d, V, K, kmax = 8, 8192, 128256, 4, 10
+    """M = 128 rows of 70B-shaped heads need more scratch than the array holds."""
+    M, d, V, K, kmax = 128, 8192, 128256, 4, 10
     assert md.heads_workspace_bytes(M, d, V, K, kmax) > (8 << 20)
     h = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
     W1 = torch.empty((K, d, d), dtype=torch.bfloat16, device="cuda")
