@@ -254,30 +254,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sb = tS + lane_off + uint32_t((c & 1) * kBN + half * kHalf);
       const int key0 = (c_begin + c) * kBN + half * kHalf;
       const bool plain = key0 + kHalf <= P;      // every key of this half is in the prefix
-      // pass 1: masked chunk maximum of this half, exchanged with the partner warp
+      // this half of the row's scores: one 64-column TMEM load, kept for both passes
+      float s[kHalf];
       float mx = -INFINITY;
       if (ok) {
+        tmem_ld64(sb, s);
+        if (plain) {
 #pragma unroll
-        for (int c32 = 0; c32 < kHalf; c32 += 32) {
-          float s[32];
-          tmem_ld32(sb + c32, s);
-          if (plain) {
+          for (int j = 0; j < kHalf; ++j) mx = fmaxf(mx, s[j]);
+        } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, s[j]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int slot = key0 + c32 + j;
-              const bool vis = slot < P || (slot < nkeys && live && tree_visible(tp, t, slot - P));
-              if (vis) mx = fmaxf(mx, s[j]);
-            }
+          for (int j = 0; j < kHalf; ++j) {
+            const int slot = key0 + j;
+            const bool vis = slot < P || (slot < nkeys && live && tree_visible(tp, t, slot - P));
+            s[j] = vis ? s[j] : -INFINITY;
+            mx = fmaxf(mx, s[j]);
           }
         }
       }
+      // exchange the half maxima with the partner warp (same lane quarter)
       xmax[half * kBM + r] = mx;
-      named_bar_sync(1, kSoftWarps * 32);
+      named_bar_sync(1 + q, 64);
       mx = fmaxf(mx, xmax[(half ^ 1) * kBM + r]);
-      named_bar_sync(1, kSoftWarps * 32);        // both halves have read before the slots are reused
+      named_bar_sync(1 + q, 64);                 // both have read before the slots are reused
       mx = (mx == -INFINITY) ? -INFINITY : mx * sc;
       // The previous P V must be done before P is overwritten or O rescaled.
       if (ok && c >= 1 && !mbar_wait(smem_u32(o_full), (c - 1) & 1)) ok = false;
@@ -299,26 +298,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       run_l *= fold;
       run_m = m_new;
-      // pass 2: P = exp2(S*scale - m) as bf16 hi + lo into swizzled smem (K-major over keys)
-      const bool none = run_m == -INFINITY;      // no visible key yet: every weight is 0
-      const float mb = none ? 0.f : run_m;
+      // P = exp2(S*scale - m) as bf16 hi + lo into swizzled smem (K-major over keys);
+      // masked keys hold -inf and give exactly 0
+      const float mb = (run_m == -INFINITY) ? 0.f : run_m;
       float sum = 0.f;
 #pragma unroll
       for (int c32 = 0; c32 < kHalf; c32 += 32) {
-        float s[32];
-        tmem_ld32(sb + c32, s);
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          float p0 = exp2f(fmaf(s[j], sc, -mb));
-          float p1 = exp2f(fmaf(s[j + 1], sc, -mb));
-          if (!plain) {
-            const int slot = key0 + c32 + j;
-            const bool v0 = slot < P || (slot < nkeys && live && tree_visible(tp, t, slot - P));
-            const bool v1 = slot + 1 < P || (slot + 1 < nkeys && live && tree_visible(tp, t, slot + 1 - P));
-            p0 = (v0 && !none) ? p0 : 0.f;
-            p1 = (v1 && !none) ? p1 : 0.f;
-          }
+          const float p0 = exp2f(fmaf(s[c32 + j], sc, -mb));
+          const float p1 = exp2f(fmaf(s[c32 + j + 1], sc, -mb));
           sum += p0 + p1;
           const uint32_t h2 = pack_bf16x2(p0, p1);
           ph[j >> 1] = h2;
@@ -364,15 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) set_status(MD_DEV_TIMEOUT);
     xmax[half * kBM + r] = run_l;
-    named_bar_sync(1, kSoftWarps * 32);
+    named_bar_sync(1 + q, 64);
     if (half == 0)
       a.part_ml[prow] = make_float2((ok && nch > 0) ? run_m : -INFINITY, run_l + xmax[kBM + r]);
 
     // The last CTA of this (request, KV head, row tile) merges the splits in order.
     __threadfence();
-    named_bar_sync(1, kSoftWarps * 32);
+    named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
     if (sw == 0 && lane == 0) *last_flag = (atomicAdd(&a.counters[tile], 1) == a.splits - 1);
-    named_bar_sync(1, kSoftWarps * 32);
+    named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
     if (*last_flag && live && half == 0) {
       __threadfence();
       const int g = grow - t * a.G;
