@@ -370,6 +370,35 @@ def run_medusa(args, w):
     ms_per_step = total_ms / args.steps
     value = job_value(world, args.steps, total_ms)
 
+    # ---- the same step replayed from CUDA graphs (one per buffer set) -------
+    graph_ms = None
+    try:
+        if world > 1:   # every rank must take the same collective steps: eager only
+            raise RuntimeError("multi-rank run")
+        graphs = []
+        for i in range(nsets):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                one_step(i)
+            graphs.append(g)
+        for i in range(args.warmup):
+            graphs[i % nsets].replay()
+        barrier()
+        torch.cuda.synchronize()
+        gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gs.record(stream)
+            for i in range(args.steps):
+                graphs[i % nsets].replay()
+            ge.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        graph_ms = slowest_rank_ms(gs.elapsed_time(ge), world, dev) / args.steps
+        del graphs
+    except Exception as exc:  # capture not possible here: report the eager number only
+        print(f"cuda graph replay unavailable: {exc}", file=sys.stderr)
+        torch.cuda.synchronize()
+
     # ---- end to end through the public API with host buffers ---------------
     e2e = None
     if not args.no_e2e:
@@ -406,6 +435,9 @@ def run_medusa(args, w):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, P),
             "roofline": roof,
+            "graph_replay": None if graph_ms is None else {
+                "ms_per_step": graph_ms, "steps_per_s": job_value(world, 1, graph_ms),
+                "note": "the same four calls captured once per buffer set in CUDA graphs and replayed"},
             "step_gbs": step_bytes / (ms_per_step / 1000.0) / 1e9 / 1.0,
             "step_gbs_frac": step_bytes / (ms_per_step / 1000.0) / 1e9 / peaks["hbm_gbs"],
             "per_call_ms": {"medusa_heads": heads_ms, "tree_build": float(per_call[:, 1].mean()),
@@ -413,7 +445,7 @@ def run_medusa(args, w):
             "attention": {"bytes": ab, "flops": af, "gbs": ab / (attn_ms / 1000) / 1e9,
                           "tflops": af / (attn_ms / 1000) / 1e12},
             "accept": {"bytes": accept_bytes(w), "gbs": accept_bytes(w) / (acc_ms / 1000) / 1e9},
-            "gpu_launches": 8 * args.steps,
+            "gpu_launches": (3 + 1 + (1 if (128 % (w.Hq // w.Hkv)) == 0 else 2) + 2) * args.steps,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -460,6 +492,17 @@ def run_part(args, w):
                 for i in range(nsets)]
         call = lambda i: step.attention(*sets[i % nsets], prefix)                # noqa: E731
         nbytes, nflops, launches = attention_bytes(w, P), attention_flops(w, P), 2
+    elif args.part == "commit":
+        tokens = synth.synthetic_tree_tokens(seed, w.B, np.array(step.tree.parent), w.V)
+        logits = synth.planted_logits_device(seed, np.array(step.tree.parent), tokens, w.V, w.accept,
+                                             sigma=w.logit_sigma, bump=w.bump, device=dev)
+        step.tokens.copy_(torch.from_numpy(tokens))
+        step.accept(logits)
+        kc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed, "k_cache", 1.0)
+        vc = sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed, "v_cache", 1.0)
+        call = lambda i: step.commit(kc, vc, prefix)                               # noqa: E731
+        nbytes = int(2 * 2 * w.B * w.Hkv * (step.accept_len.sum().item() + w.B) * w.dh * 2)
+        nflops, launches = 0, 1
     else:
         tokens = synth.synthetic_tree_tokens(seed, w.B, np.array(step.tree.parent), w.V)
         logits = synth.planted_logits(seed, np.array(step.tree.parent), tokens, w.V, w.accept,
@@ -473,17 +516,34 @@ def run_part(args, w):
         for i in range(args.warmup):
             call(i)
     stream.synchronize()
+    # Replay the calls from a CUDA graph so that host-side launch overhead does
+    # not show up between short kernels; fall back to eager launches.
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
+            for i in range(args.steps):
+                call(i)
+        graph.replay()
+        stream.synchronize()
+    except Exception:
+        graph = None
+        torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         start.record(stream)
-        for i in range(args.steps):
-            call(i)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                call(i)
         end.record(stream)
     torch.cuda.synchronize()
     status = md.device_status(stream=stream)
     ms = start.elapsed_time(end) / args.steps
     peaks = measured_peaks()
     print(json.dumps({"part": args.part, "workload": w.name, "ms_per_call": ms, "calls": args.steps,
+                      "launch": "cuda-graph replay" if graph is not None else "eager",
                       "gbs": nbytes / (ms / 1000) / 1e9, "hbm_frac": nbytes / (ms / 1000) / 1e9 / peaks["hbm_gbs"],
                       "tflops": nflops / (ms / 1000) / 1e12 if nflops else None,
                       "algorithmic_bytes": nbytes, "flops": nflops, "gpu_launches": launches * args.steps,
@@ -637,7 +697,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["medusa", "reference"], default="medusa")
     ap.add_argument("--workload", default="llama3-70b", choices=sorted(WORKLOADS))
-    ap.add_argument("--part", choices=["step", "heads", "attention", "accept"], default="step",
+    ap.add_argument("--part", choices=["step", "heads", "attention", "accept", "commit"], default="step",
                     help="time one call alone (profiling); the JSON line then reports that call only")
     ap.add_argument("--sweep", action="store_true",
                     help="run the 8B-shaped sweep (B x tree x prefix x rule), one JSON line per point")

@@ -66,7 +66,9 @@ enum {
   MD_DEV_BAD_PREFIX = 1,   /* prefix_len[b] < 0 or prefix_len[b] + T > S_max     */
   MD_DEV_BAD_ROW = 2,      /* head_row[b] outside [0, M)                         */
   MD_DEV_BAD_TOKEN = 4,    /* a token id outside [0, V) reached tree_accept      */
-  MD_DEV_TIMEOUT = 8       /* a pipeline wait exceeded its bound                 */
+  MD_DEV_TIMEOUT = 8,      /* a pipeline wait exceeded its bound                 */
+  MD_DEV_BAD_PATH = 16     /* md_tree_commit got a length or path that is not a  */
+                           /* root-to-node path of the tree                       */
 };
 
 /* Supported ranges (anything else: MD_ERR_UNSUPPORTED).
@@ -265,6 +267,35 @@ MD_API md_status md_tree_accept(const float* logits, int32_t V, const int32_t* t
                          int32_t B, int32_t K, int32_t mode, float temperature, float eps, float alpha,
                          int32_t* accept_len, int32_t* path, int32_t* bonus, void* ws, size_t ws_bytes,
                          void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 5. Advancing along the accepted branch.                                   */
+/* ------------------------------------------------------------------------ */
+
+/* KV compaction and the next step's inputs, after md_tree_accept.
+ * Source: "Medusa heads versus separate draft model", section "Acceptance",
+ * tree paragraph ("if any branch matches, the step advances along it").
+ *
+ * For request b with P = prefix_len[b], L = accept_len[b], path = path[b]:
+ *   K/V slot P + i  <-  K/V slot P + path[i]      (i = 0..L, in place; other
+ *                                                  slots are left unchanged)
+ *   new_prefix_len[b] = P + L + 1    (the root and the L accepted tokens)
+ *   next_root[b]      = bonus[b]
+ *   next_head_row[b]  = b * T + path[L]   (row of the last accepted node when
+ *                                          the heads ran on all B * T nodes)
+ *
+ * k_cache, v_cache [B, Hkv, S_max, dh] bf16 (updated in place).
+ * prefix_len [B] is read only; new_prefix_len [B] must be a different buffer.
+ * accept_len [B], path [B, K+1], bonus [B] from md_tree_accept (K = its K).
+ * A length or path that is not a root-to-node path of the tree, or a prefix
+ * that does not fit, sets MD_DEV_BAD_PATH and leaves that request's cache
+ * unchanged (new_prefix_len = P, next_head_row = -1).
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED (dh not 64/128), MD_ERR_CUDA. */
+MD_API md_status md_tree_commit(md_bf16* k_cache, md_bf16* v_cache, int32_t S_max, int32_t Hkv, int32_t dh,
+                                const md_tree* tree, int32_t B, const int32_t* prefix_len,
+                                const int32_t* accept_len, const int32_t* path, int32_t K, const int32_t* bonus,
+                                int32_t* new_prefix_len, int32_t* next_root, int32_t* next_head_row,
+                                void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Status.                                                                   */

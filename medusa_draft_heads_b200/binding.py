@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(HERE, "libmedusa.so")
 
 MD_ACCEPT_GREEDY = 0
 MD_ACCEPT_TYPICAL = 1
-DEV_BAD_PREFIX, DEV_BAD_ROW, DEV_BAD_TOKEN, DEV_TIMEOUT = 1, 2, 4, 8
+DEV_BAD_PREFIX, DEV_BAD_ROW, DEV_BAD_TOKEN, DEV_TIMEOUT, DEV_BAD_PATH = 1, 2, 4, 8, 16
 
 _lib = None
 _P = ctypes.c_void_p
@@ -37,6 +37,7 @@ _SIGNATURES = {
     "md_tree_attention": [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P],
     "md_accept_workspace": [_I, _I, _I, ctypes.POINTER(_SZ)],
     "md_tree_accept": [_P, _I, _P, _P, _I, _I, _I, _F, _F, _F, _P, _P, _P, _P, _SZ, _P],
+    "md_tree_commit": [_P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
     "md_get_device_status": [_P, ctypes.POINTER(_I), _I],
     "md_status_string": [_I],
     "md_version": [],
@@ -223,6 +224,25 @@ def tree_accept(logits, tokens, tree: Tree, accept_len, path, bonus, ws, mode="g
         _ptr(path, torch.int32, "path", 2), _ptr(bonus, torch.int32, "bonus"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream))
     _check(rc, "md_tree_accept")
+
+
+def tree_commit(k_cache, v_cache, tree: Tree, prefix_len, accept_len, path, bonus, new_prefix_len, next_root,
+                next_head_row, stream=None):
+    """md_tree_commit: move the accepted path's K/V next to the prefix (in place)
+    and produce the next step's prefix lengths, root tokens and head rows."""
+    B, Hkv, S_max, dh = k_cache.shape
+    K = path.shape[1] - 1
+    _same("tree_commit", v_cache=(tuple(v_cache.shape), (B, Hkv, S_max, dh)), path_rows=(path.shape[0], B),
+          prefix_len=(tuple(prefix_len.shape), (B,)), accept_len=(tuple(accept_len.shape), (B,)),
+          bonus=(tuple(bonus.shape), (B,)), new_prefix_len=(tuple(new_prefix_len.shape), (B,)),
+          next_root=(tuple(next_root.shape), (B,)), next_head_row=(tuple(next_head_row.shape), (B,)))
+    rc = lib().md_tree_commit(
+        _ptr(k_cache, torch.bfloat16, "k_cache", 4), _ptr(v_cache, torch.bfloat16, "v_cache", 4), S_max, Hkv, dh,
+        tree.handle, B, _ptr(prefix_len, torch.int32, "prefix_len"), _ptr(accept_len, torch.int32, "accept_len"),
+        _ptr(path, torch.int32, "path", 2), K, _ptr(bonus, torch.int32, "bonus"),
+        _ptr(new_prefix_len, torch.int32, "new_prefix_len"), _ptr(next_root, torch.int32, "next_root"),
+        _ptr(next_head_row, torch.int32, "next_head_row"), _stream(stream))
+    _check(rc, "md_tree_commit")
 
 
 def device_status(clear: bool = True, stream=None) -> int:

@@ -15,6 +15,7 @@
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "accept.cuh"
+#include "commit.cuh"
 
 struct md_tree {
   md::TreeParams tp;
@@ -619,6 +620,25 @@ md_status md_tree_accept(const float* logits, int32_t V, const int32_t* tokens, 
       MD_OK)
     return s;
   return launch_pdl(md::acc::accept_walk_kernel, dim3(B), dim3(MD_MAX_T), 0, st, tree->tp, a);
+}
+
+md_status md_tree_commit(md_bf16* k_cache, md_bf16* v_cache, int32_t S_max, int32_t Hkv, int32_t dh,
+                         const md_tree* tree, int32_t B, const int32_t* prefix_len, const int32_t* accept_len,
+                         const int32_t* path, int32_t K, const int32_t* bonus, int32_t* new_prefix_len,
+                         int32_t* next_root, int32_t* next_head_row, void* stream) {
+  if (!k_cache || !v_cache || !tree || !prefix_len || !accept_len || !path || !bonus || !new_prefix_len ||
+      !next_root || !next_head_row)
+    return MD_ERR_INVALID_ARG;
+  if (B < 1 || Hkv < 1 || S_max < tree->tp.T || K < tree->tp.max_depth || K > MD_MAX_K) return MD_ERR_INVALID_ARG;
+  if (dh != 64 && dh != 128) return MD_ERR_UNSUPPORTED;
+  if (new_prefix_len == prefix_len || !aligned(k_cache, 16) || !aligned(v_cache, 16)) return MD_ERR_INVALID_ARG;
+  md::commit::Args a;
+  a.kc = k_cache; a.vc = v_cache; a.prefix_len = prefix_len; a.accept_len = accept_len; a.path = path;
+  a.bonus = bonus; a.new_prefix_len = new_prefix_len; a.next_root = next_root; a.next_head_row = next_head_row;
+  a.S_max = S_max; a.Hkv = Hkv; a.dh = dh; a.K = K;
+  const int smem = 2 * (MD_MAX_K + 1) * dh * 2;
+  return launch_pdl(md::commit::tree_commit_kernel, dim3(Hkv, B), dim3(md::commit::kThreads), smem,
+                    static_cast<cudaStream_t>(stream), tree->tp, a);
 }
 
 md_status md_get_device_status(void* stream, int32_t* out, int32_t clear) {

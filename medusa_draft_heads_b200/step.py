@@ -9,7 +9,7 @@ from __future__ import annotations
 import torch
 
 from .binding import (Tree, accept_workspace_bytes, attention_workspace_bytes, heads_workspace_bytes,
-                      medusa_heads, tree_accept, tree_attention, tree_build, workspace)
+                      medusa_heads, tree_accept, tree_attention, tree_build, tree_commit, workspace)
 from .tree_spec import tree_arrays
 
 
@@ -38,6 +38,9 @@ class MedusaStep:
         self.accept_len = torch.empty((B,), **i32)
         self.path = torch.empty((B, K + 1), **i32)
         self.bonus = torch.empty((B,), **i32)
+        self.new_prefix_len = torch.empty((B,), **i32)
+        self.next_root = torch.empty((B,), **i32)
+        self.next_head_row = torch.empty((B,), **i32)
         self.ws_heads = workspace(heads_workspace_bytes(M, d, V, K, self.kmax), dev)
         self.ws_attn = workspace(attention_workspace_bytes(B, self.T, Hq, Hkv, dh, S_max), dev)
         self.ws_acc = workspace(accept_workspace_bytes(B, self.T, V), dev)
@@ -56,6 +59,10 @@ class MedusaStep:
     def accept(self, logits, stream=None):
         tree_accept(logits, self.tokens, self.tree, self.accept_len, self.path, self.bonus, self.ws_acc,
                     mode=self.mode, temperature=self.temperature, eps=self.eps, alpha=self.alpha, stream=stream)
+
+    def commit(self, k_cache, v_cache, prefix_len, stream=None):
+        tree_commit(k_cache, v_cache, self.tree, prefix_len, self.accept_len, self.path, self.bonus,
+                    self.new_prefix_len, self.next_root, self.next_head_row, stream=stream)
 
     def run(self, h, W1, b1, Wv, root_token, prefix_len, q, k_cache, v_cache, logits, head_row=None,
             stream=None):
