@@ -47,8 +47,7 @@ L2_BYTES = 126 * 1024 * 1024
 # Algorithmic byte and flop counts (what the method must move / compute).
 # --------------------------------------------------------------------------- #
 def heads_bytes(w):
-    weights = 2 * w.K * (w.d * w.d + w.d + w.d * w.V)
-    return weights + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax
+    return w.head_weight_bytes() + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax
 
 
 def slowest_rank_ms(ms: float, world: int, device=None) -> float:
@@ -288,7 +287,8 @@ def run_medusa(args, w):
     bf = dict(dtype=torch.bfloat16, device=dev)
     W1 = sdev.fill_normal(torch.empty((w.K, w.d, w.d), **bf), seed, "W1", w.w_sigma)
     b1 = sdev.fill_normal(torch.empty((w.K, w.d), **bf), seed, "b1", w.w_sigma)
-    Wv = sdev.fill_normal(torch.empty((w.K, w.d, w.V), **bf), seed, "Wv", w.w_sigma)
+    Wv = sdev.fill_normal(torch.empty(((w.d, w.V) if w.shared_vocab else (w.K, w.d, w.V)), **bf), seed, "Wv",
+                          w.w_sigma)
     h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), seed, "h", 1.0)
     root = torch.from_numpy(synth.root_tokens(seed, w.B, w.V)).to(dev)
     P = synth.prefix_lengths(seed, w.B, *w.prefix)
@@ -296,7 +296,7 @@ def run_medusa(args, w):
     tups = md.select_tree(w.k_per_head, w.accept, w.n_nodes)
     step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
                       Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
-                      alpha=w.alpha, device=dev)
+                      alpha=w.alpha, device=dev, shared_vocab=w.shared_vocab)
     head_row = None
     if w.M != w.B:
         head_row = torch.arange(w.B, dtype=torch.int32, device=dev) * w.T
@@ -474,16 +474,17 @@ def run_part(args, w):
     tups = md.select_tree(w.k_per_head, w.accept, w.n_nodes)
     step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
                       Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
-                      alpha=w.alpha, device=dev)
+                      alpha=w.alpha, device=dev, shared_vocab=w.shared_vocab)
     P = synth.prefix_lengths(seed, w.B, *w.prefix)
     prefix = torch.from_numpy(P).to(dev)
     if args.part == "heads":
         W1 = sdev.fill_normal(torch.empty((w.K, w.d, w.d), **bf), seed, "W1", w.w_sigma)
         b1 = sdev.fill_normal(torch.empty((w.K, w.d), **bf), seed, "b1", w.w_sigma)
-        Wv = sdev.fill_normal(torch.empty((w.K, w.d, w.V), **bf), seed, "Wv", w.w_sigma)
+        Wv = sdev.fill_normal(torch.empty(((w.d, w.V) if w.shared_vocab else (w.K, w.d, w.V)), **bf), seed, "Wv",
+                              w.w_sigma)
         h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), seed, "h", 1.0)
         call = lambda i: step.heads(h, W1, b1, Wv)                              # noqa: E731
-        nbytes, nflops, launches = heads_bytes(w), 2 * w.M * w.K * w.d * (w.d + w.V), 3
+        nbytes, nflops, launches = heads_bytes(w), heads_flops(w), 3
     elif args.part == "attention":
         nsets = 8
         sets = [(sdev.fill_normal(torch.empty((w.B, w.T, w.Hq, w.dh), **bf), seed + i, "q", 1.0),
@@ -516,34 +517,36 @@ def run_part(args, w):
         for i in range(args.warmup):
             call(i)
     stream.synchronize()
-    # Replay the calls from a CUDA graph so that host-side launch overhead does
-    # not show up between short kernels; fall back to eager launches.
-    graph = None
+    def timed(fn):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            fn()
+            end.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / args.steps
+
+    def eager():
+        for i in range(args.steps):
+            call(i)
+
+    ms = timed(eager)
+    # The same calls replayed from one CUDA graph (no host launch overhead).
+    graph_ms = None
     try:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
-            for i in range(args.steps):
-                call(i)
+            eager()
         graph.replay()
         stream.synchronize()
+        graph_ms = timed(graph.replay)
+        del graph
     except Exception:
-        graph = None
         torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            for i in range(args.steps):
-                call(i)
-        end.record(stream)
-    torch.cuda.synchronize()
     status = md.device_status(stream=stream)
-    ms = start.elapsed_time(end) / args.steps
     peaks = measured_peaks()
     print(json.dumps({"part": args.part, "workload": w.name, "ms_per_call": ms, "calls": args.steps,
-                      "launch": "cuda-graph replay" if graph is not None else "eager",
+                      "graph_ms_per_call": graph_ms,
                       "gbs": nbytes / (ms / 1000) / 1e9, "hbm_frac": nbytes / (ms / 1000) / 1e9 / peaks["hbm_gbs"],
                       "tflops": nflops / (ms / 1000) / 1e12 if nflops else None,
                       "algorithmic_bytes": nbytes, "flops": nflops, "gpu_launches": launches * args.steps,

@@ -146,6 +146,27 @@ MD_API md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_b
                           int32_t kmax, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* Workspace bytes md_medusa_heads_shared needs for these sizes. */
+MD_API md_status md_heads_shared_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax, size_t* bytes);
+
+/* The K heads with ONE vocabulary projection shared by all of them.
+ * Source: "Medusa heads versus separate draft model", section "What
+ * interviewers probe next": each head normally has its own d x V projection
+ * (initialised from the LM head); sharing one saves (K - 1) d V parameters
+ * (3.15B for four heads at d = 8,192, V = 128,256) at some cost to
+ * acceptance. The residual blocks stay per head:
+ *   z[m,k,:]     = bf16_rne( h[m,:] + SiLU(h[m,:] W1[k] + b1[k]) )
+ *   logit[m,k,v] = sum_i z[m,k,i] * Wv[i,v]
+ * and the top-k is as in md_medusa_heads. Arguments as md_medusa_heads except
+ * Wv [d, V] bf16 (16-byte aligned, as are h and b1). The projection is
+ * streamed once for all heads: 2 d V bytes instead of 2 K d V.
+ * Errors: as md_medusa_heads. */
+MD_API md_status md_medusa_heads_shared(const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
+                                        const md_bf16* Wv, int32_t M, int32_t d, int32_t V, int32_t K,
+                                        const int32_t* k_per_head, int32_t kmax, int32_t* topk_ids,
+                                        float* topk_vals, float* logits_dbg, void* ws, size_t ws_bytes,
+                                        void* stream);
+
 /* Size of the library-owned scratch behind md_medusa_heads_static (8 MiB). */
 #define MD_HEADS_STATIC_SCRATCH_BYTES (8u << 20)
 

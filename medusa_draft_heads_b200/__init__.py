@@ -11,6 +11,7 @@ The kernels live in ``libmedusa.so`` (built from ``csrc/`` for sm_100a); this
 package only marshals arguments to it.
 """
 from .binding import (MedusaError, Tree, accept_workspace_bytes, attention_workspace_bytes,  # noqa: F401
-                      device_status, heads_workspace_bytes, lib, medusa_heads, tree_accept, tree_attention,
+                      device_status, heads_shared_workspace_bytes, heads_workspace_bytes, lib, medusa_heads,
+                      medusa_heads_shared, tree_accept, tree_attention,
                       tree_build, tree_commit, version, workspace)
 from .tree_spec import select_tree, tree_arrays  # noqa: F401

@@ -32,6 +32,8 @@ _SIGNATURES = {
     "md_tree_info": [_P, ctypes.POINTER(_I), ctypes.POINTER(_I)],
     "md_heads_workspace": [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
     "md_medusa_heads": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
+    "md_heads_shared_workspace": [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
+    "md_medusa_heads_shared": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
     "md_tree_build": [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
     "md_attention_workspace": [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
     "md_tree_attention": [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P],
@@ -140,6 +142,12 @@ def heads_workspace_bytes(M, d, V, K, kmax) -> int:
     return n.value
 
 
+def heads_shared_workspace_bytes(M, d, V, K, kmax) -> int:
+    n = _SZ()
+    _check(lib().md_heads_shared_workspace(M, d, V, K, kmax, ctypes.byref(n)), "md_heads_shared_workspace")
+    return n.value
+
+
 def attention_workspace_bytes(B, T, Hq, Hkv, dh, S_max) -> int:
     n = _SZ()
     _check(lib().md_attention_workspace(B, T, Hq, Hkv, dh, S_max, ctypes.byref(n)), "md_attention_workspace")
@@ -174,6 +182,26 @@ def medusa_heads(h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, ws, logits_dbg=
         _ptr(topk_ids, torch.int32, "topk_ids", 3), _ptr(topk_vals, torch.float32, "topk_vals", 3),
         _ptr(logits_dbg, torch.float32, "logits_dbg", 3), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(rc, "md_medusa_heads")
+
+
+def medusa_heads_shared(h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, ws, logits_dbg=None, stream=None):
+    """md_medusa_heads_shared: h [M,d], W1 [K,d,d], b1 [K,d], ONE Wv [d,V] bf16 ->
+    topk_ids [M,K,kmax] int32, topk_vals [M,K,kmax] fp32."""
+    M, d = h.shape
+    K = W1.shape[0]
+    V = Wv.shape[1]
+    kmax = topk_ids.shape[2]
+    _same("medusa_heads_shared", W1=(tuple(W1.shape), (K, d, d)), b1=(tuple(b1.shape), (K, d)),
+          Wv=(tuple(Wv.shape), (d, V)), topk_ids=(tuple(topk_ids.shape), (M, K, kmax)),
+          topk_vals=(tuple(topk_vals.shape), (M, K, kmax)), k_per_head=(len(k_per_head), K))
+    if logits_dbg is not None:
+        _same("medusa_heads_shared", logits_dbg=(tuple(logits_dbg.shape), (M, K, V)))
+    rc = lib().md_medusa_heads_shared(
+        _ptr(h, torch.bfloat16, "h", 2), _ptr(W1, torch.bfloat16, "W1", 3), _ptr(b1, torch.bfloat16, "b1", 2),
+        _ptr(Wv, torch.bfloat16, "Wv", 2), M, d, V, K, _host_i32(k_per_head), kmax,
+        _ptr(topk_ids, torch.int32, "topk_ids", 3), _ptr(topk_vals, torch.float32, "topk_vals", 3),
+        _ptr(logits_dbg, torch.float32, "logits_dbg", 3), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "md_medusa_heads_shared")
 
 
 def tree_build(tree: Tree, topk_ids, root_token, prefix_len, tokens, parent, anc, pos, head_row=None,

@@ -92,6 +92,7 @@ struct W1Args {
   float* part;         // [splits, K, M, d]
   int* counters;       // [K, ntile_o]
   int d, K, splits, rows, ntile_o;
+  int shared;          // 1: one projection for all heads: z row (m, k) goes to slot m*K + k of zt[0]
 };
 
 template <int M>
@@ -209,9 +210,14 @@ __global__ void __launch_bounds__(kW1Threads) heads_w1_kernel(W1Args a) {
         zv[m] = 0;
       }
     }
-    reinterpret_cast<uint4*>(a.zt)[size_t(k) * d + col] =
-        make_uint4(zv[0] | (uint32_t(zv[1]) << 16), zv[2] | (uint32_t(zv[3]) << 16), zv[4] | (uint32_t(zv[5]) << 16),
-                   zv[6] | (uint32_t(zv[7]) << 16));
+    if (a.shared) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) a.zt[size_t(col) * kZPad + m * a.K + k] = zv[m];
+    } else {
+      reinterpret_cast<uint4*>(a.zt)[size_t(k) * d + col] =
+          make_uint4(zv[0] | (uint32_t(zv[1]) << 16), zv[2] | (uint32_t(zv[3]) << 16),
+                     zv[4] | (uint32_t(zv[5]) << 16), zv[6] | (uint32_t(zv[7]) << 16));
+    }
   }
   if (t == 0) a.counters[k * a.ntile_o + ct] = 0;
 }
@@ -233,6 +239,7 @@ struct VocabArgs {
   int* cand_id;
   float* logits_dbg;   // [M, K, V] or null
   int d, V, K, kmax, ntiles, units, nstages;
+  int shared, kh;      // shared projection: K == 1 and row m is (m / kh, head m % kh)
   int kph[MD_MAX_K];
 };
 
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       }
       float pv = INFINITY;
       int pid = -1;
-      const int kk = a.kph[k];
+      const int kk = a.shared ? a.kph[m % a.kh] : a.kph[k];
       float nrv = -INFINITY;
       int nri = INT_MAX;
       for (int r = 0; r < kk; ++r) {
@@ -459,6 +466,7 @@ struct MergeArgs {
   float* topk_vals;
   int K, kmax, nslots;
   int partitioned, units, ntiles, mrows;   // producer partition (partitioned == 1)
+  int kh;              // heads for the top-k size: row mk uses kph[mk % kh]
   int kph[MD_MAX_K];
 };
 
@@ -528,7 +536,7 @@ __global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
   __shared__ int wi[8][kListMax];
   const int mk = blockIdx.x;
   const int k = mk % a.K, m = mk / a.K;
-  const int kk = a.kph[k];
+  const int kk = a.kph[mk % a.kh];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t base = size_t(mk) * a.nslots * a.kmax;
   const long long run = (long long)(m / a.mrows) * a.K + k;   // (row tile, head) run of (m, k)

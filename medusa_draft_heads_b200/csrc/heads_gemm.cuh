@@ -55,6 +55,8 @@ struct Args {
   int* cand_id;
   float* logits_dbg;              // [M, K, N] or null
   int kmax;
+  int zg_mk;                      // phase 1: write z rows in (row, head) order [M*K, d]
+  int kh;                         // phase 2: row m uses kph[m % kh] when K == 1 (shared projection)
   int kph[MD_MAX_K];
 };
 
@@ -225,7 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (live && o0 < a.d) {
             const uint4* hp = reinterpret_cast<const uint4*>(a.h + size_t(m) * a.d + o0);
             const uint4* bp = reinterpret_cast<const uint4*>(a.b1 + size_t(k) * a.d + o0);
-            uint4* zp = reinterpret_cast<uint4*>(a.zg + (size_t(k) * a.M + m) * a.d + o0);
+            uint4* zp = reinterpret_cast<uint4*>(
+                a.zg + (a.zg_mk ? size_t(m) * a.K + k : size_t(k) * a.M + m) * a.d + o0);
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const uint4 hv = hp[g], bv = __ldg(bp + g);
@@ -246,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         if (k != cur_k) {         // a new (row tile, head) run starts: fresh lists
-          L.kk = a.kph[k];
+          L.kk = a.kh > 0 ? a.kph[m % a.kh] : a.kph[k];
           L.reset();
           cur_k = k;
         }

@@ -125,6 +125,7 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   wa.part = reinterpret_cast<float*>(ws + pl.off_part);
   wa.counters = reinterpret_cast<int*>(ws + pl.off_cnt);
   wa.d = pl.d; wa.K = pl.K; wa.splits = pl.splits; wa.rows = pl.rows; wa.ntile_o = pl.ntile_o;
+  wa.shared = 0;
   if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, size_t(pl.K) * pl.ntile_o * 4, st))) != MD_OK) return s;
   const int w1_smem = pl.rows * 16 + kConsumerWarps * M * kW1TileO * 4;
   if ((s = set_smem(heads_w1_kernel<M>, w1_smem)) != MD_OK) return s;
@@ -141,6 +142,7 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   va.logits_dbg = logits_dbg;
   va.d = pl.d; va.V = pl.V; va.K = pl.K; va.kmax = pl.kmax; va.ntiles = pl.ntiles; va.units = pl.units;
   va.nstages = pl.nstages;
+  va.shared = 0; va.kh = pl.K;
   for (int k = 0; k < MD_MAX_K; ++k) va.kph[k] = k < pl.K ? kph[k] : 0;
   const int v_smem = vocab_smem_bytes(M, pl.nstages);
   if ((s = set_smem(heads_vocab_kernel<M>, v_smem)) != MD_OK) return s;
@@ -161,7 +163,7 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = pl.K; ma.kmax = pl.kmax; ma.nslots = pl.grid;
-  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.mrows = 1 << 30;
+  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.mrows = 1 << 30; ma.kh = pl.K;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
   return launch_pdl(heads_merge_kernel, dim3(pl.M * pl.K), dim3(256), 0, st, ma);
 }
@@ -258,9 +260,130 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = K; ma.kmax = kmax; ma.nslots = pl.grid2;
-  ma.partitioned = 1; ma.units = K * pl.ntiles2 * pl.mtiles; ma.ntiles = pl.ntiles2; ma.mrows = kBM;
+  ma.partitioned = 1; ma.units = K * pl.ntiles2 * pl.mtiles; ma.ntiles = pl.ntiles2; ma.mrows = kBM; ma.kh = K;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
   return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
+}
+
+// ------------------- shared vocabulary projection (one Wv) -------------------
+// Phase 1 is the per-head residual block; phase 2 treats the M*K rows
+// (m, k) -> m*K + k as rows of one head against the single projection.
+
+struct SharedPlan {
+  bool stream;                 // M*K <= 4: CUDA-core weight stream; else tensor cores
+  md::heads::Plan p1, p2;      // streaming: phase-1 plan (M rows, K heads), phase-2 plan (M*K rows, 1 head)
+  GemmPlan g1, g2;             // tensor cores: phase 1 (M rows, K heads), phase 2 (M*K rows, 1 head)
+  size_t off2, bytes;
+};
+
+SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
+  using md::heads::align256;
+  SharedPlan p{};
+  p.stream = M * K <= md::heads::kMaxM;
+  if (p.stream) {
+    p.p1 = md::heads::make_plan(M, d, V, K, kmax, num_sms());
+    p.p2 = md::heads::make_plan(M * K, d, V, 1, kmax, num_sms());
+    p.off2 = align256(p.p1.off_cval);                    // phase-2 candidates after phase-1 data
+    p.bytes = p.off2 + (p.p2.bytes - p.p2.off_cval);
+  } else {
+    p.g1 = gemm_plan(M, d, V, K, kmax);                   // z [M*K, d] lives at g1.off_z
+    p.g2 = gemm_plan(M * K, d, V, 1, kmax);
+    p.off2 = align256(p.g1.off_z + size_t(K) * M * d * 2);
+    p.bytes = p.off2 + (p.g2.bytes - p.g2.off_cval);
+  }
+  return p;
+}
+
+template <int MK>
+md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16* h, const md_bf16* W1,
+                                     const md_bf16* b1, const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids,
+                                     float* topk_vals, float* logits_dbg, uint8_t* ws, cudaStream_t st) {
+  using namespace md::heads;
+  const Plan& p1 = sp.p1;
+  const Plan& p2 = sp.p2;
+  md_status s;
+  W1Args wa;
+  wa.h = h; wa.W1 = W1; wa.b1 = b1;
+  wa.zt = reinterpret_cast<uint16_t*>(ws + p1.off_zt);
+  wa.part = reinterpret_cast<float*>(ws + p1.off_part);
+  wa.counters = reinterpret_cast<int*>(ws + p1.off_cnt);
+  wa.d = p1.d; wa.K = p1.K; wa.splits = p1.splits; wa.rows = p1.rows; wa.ntile_o = p1.ntile_o;
+  wa.shared = 1;
+  if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, size_t(p1.K) * p1.ntile_o * 4, st))) != MD_OK) return s;
+  auto run_w1 = [&](auto kern, int smem) -> md_status {
+    md_status r;
+    if ((r = set_smem(kern, smem)) != MD_OK) return r;
+    kern<<<dim3(p1.ntile_o, p1.splits, p1.K), kW1Threads, smem, st>>>(wa);
+    return last_launch();
+  };
+  switch (M) {   // phase-1 rows (M * K <= 4)
+    case 1: s = run_w1(heads_w1_kernel<1>, p1.rows * 16 + kConsumerWarps * 1 * kW1TileO * 4); break;
+    case 2: s = run_w1(heads_w1_kernel<2>, p1.rows * 16 + kConsumerWarps * 2 * kW1TileO * 4); break;
+    case 3: s = run_w1(heads_w1_kernel<3>, p1.rows * 16 + kConsumerWarps * 3 * kW1TileO * 4); break;
+    case 4: s = run_w1(heads_w1_kernel<4>, p1.rows * 16 + kConsumerWarps * 4 * kW1TileO * 4); break;
+    default: return MD_ERR_UNSUPPORTED;
+  }
+  if (s != MD_OK) return s;
+  CUtensorMap map;
+  if ((s = make_map_2d(&map, Wv, uint64_t(p2.V), uint64_t(p2.d), kTileV, kStageRows)) != MD_OK) return s;
+  VocabArgs va;
+  va.zt = wa.zt;
+  va.cand_val = reinterpret_cast<float*>(ws + sp.off2);
+  va.cand_id = reinterpret_cast<int*>(ws + sp.off2 + (p2.off_cid - p2.off_cval));
+  va.logits_dbg = logits_dbg;
+  va.d = p2.d; va.V = p2.V; va.K = 1; va.kmax = p2.kmax; va.ntiles = p2.ntiles; va.units = p2.units;
+  va.nstages = p2.nstages;
+  va.shared = 1; va.kh = p1.K;
+  for (int k = 0; k < MD_MAX_K; ++k) va.kph[k] = k < p1.K ? kph[k] : 0;
+  const int v_smem = vocab_smem_bytes(MK, p2.nstages);
+  if ((s = set_smem(heads_vocab_kernel<MK>, v_smem)) != MD_OK) return s;
+  if ((s = launch_pdl(heads_vocab_kernel<MK>, dim3(p2.grid), dim3((kConsumerWarps + 1) * 32), v_smem, st, map,
+                      va)) != MD_OK)
+    return s;
+  MergeArgs ma;
+  ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
+  ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
+  ma.K = 1; ma.kmax = p2.kmax; ma.nslots = p2.grid;
+  ma.partitioned = 1; ma.units = p2.units; ma.ntiles = p2.ntiles; ma.mrows = 1 << 30; ma.kh = p1.K;
+  for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
+  return launch_pdl(heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
+}
+
+template <int KK>
+md_status launch_heads_shared_gemm(const SharedPlan& sp, int M, int d, int V, int K, int kmax, const md_bf16* h,
+                                   const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, const int32_t* kph,
+                                   int32_t* topk_ids, float* topk_vals, float* logits_dbg, uint8_t* ws,
+                                   cudaStream_t st) {
+  using namespace md::gemm;
+  md_status s;
+  const int MK = M * K;
+  Args ga = {};
+  ga.d = d; ga.kmax = kmax; ga.h = h; ga.b1 = b1;
+  ga.zg = reinterpret_cast<uint16_t*>(ws + sp.g1.off_z);
+  ga.cand_val = reinterpret_cast<float*>(ws + sp.off2);
+  ga.cand_id = reinterpret_cast<int*>(ws + sp.off2 + (sp.g2.off_cid - sp.g2.off_cval));
+  ga.logits_dbg = logits_dbg;
+  for (int k = 0; k < MD_MAX_K; ++k) ga.kph[k] = k < K ? kph[k] : 0;
+  // phase 1: per-head residual blocks, z rows written in (row, head) order
+  CUtensorMap amap, bmap;
+  if ((s = make_map_3d_sw128(&amap, h, d, M, 1, kBK, kBM)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&bmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
+  ga.M = M; ga.K = K; ga.N = d; ga.mtiles = sp.g1.mtiles; ga.ntiles = sp.g1.ntiles1;
+  ga.tiles = K * sp.g1.ntiles1 * sp.g1.mtiles; ga.a_shared = 1; ga.zg_mk = 1; ga.kh = 0;
+  if ((s = launch_gemm<EPI_SILU, KK>(amap, bmap, ga, false, st)) != MD_OK) return s;
+  // phase 2: the M*K rows against the one projection
+  if ((s = make_map_3d_sw128(&amap, ga.zg, d, MK, 1, kBK, kBM)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&bmap, Wv, V, d, 1, 64, kBK)) != MD_OK) return s;
+  ga.M = MK; ga.K = 1; ga.N = V; ga.mtiles = sp.g2.mtiles; ga.ntiles = sp.g2.ntiles2;
+  ga.tiles = sp.g2.ntiles2 * sp.g2.mtiles; ga.a_shared = 1; ga.zg_mk = 0; ga.kh = K;
+  if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, true, st)) != MD_OK) return s;
+  md::heads::MergeArgs ma;
+  ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
+  ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
+  ma.K = 1; ma.kmax = kmax; ma.nslots = sp.g2.grid2;
+  ma.partitioned = 1; ma.units = sp.g2.ntiles2 * sp.g2.mtiles; ma.ntiles = sp.g2.ntiles2; ma.mrows = kBM; ma.kh = K;
+  for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
+  return launch_pdl(md::heads::heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
 }
 
 md_status heads_check(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax) {
@@ -501,6 +624,51 @@ md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1
     case 4: return launch_heads<4>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
     default: return MD_ERR_UNSUPPORTED;
   }
+}
+
+md_status md_heads_shared_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax, size_t* bytes) {
+  if (!bytes) return MD_ERR_INVALID_ARG;
+  md_status s = heads_check(M, d, V, K, kmax);
+  if (s != MD_OK) return s;
+  if (size_t(M) * K > size_t(md::gemm::kMaxM)) return MD_ERR_UNSUPPORTED;
+  *bytes = shared_plan(M, d, V, K, kmax).bytes;
+  return MD_OK;
+}
+
+md_status md_medusa_heads_shared(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
+                                 int32_t M, int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax,
+                                 int32_t* topk_ids, float* topk_vals, float* logits_dbg, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
+  size_t need = 0;
+  md_status s = md_heads_shared_workspace(M, d, V, K, kmax, &need);
+  if (s != MD_OK) return s;
+  int mk = 0;
+  for (int k = 0; k < K; ++k) {
+    if (k_per_head[k] < 1 || k_per_head[k] > kmax || k_per_head[k] > V) return MD_ERR_INVALID_ARG;
+    mk = std::max(mk, int(k_per_head[k]));
+  }
+  if (!aligned(h, 16) || !aligned(W1, 16) || !aligned(b1, 16) || !aligned(Wv, 16) || !aligned(topk_ids, 4) ||
+      !aligned(topk_vals, 4) || (logits_dbg && !aligned(logits_dbg, 16)))
+    return MD_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  const SharedPlan sp = shared_plan(M, d, V, K, kmax);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  if (sp.stream) {
+    switch (M * K) {
+      case 1: return launch_heads_shared_stream<1>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+      case 2: return launch_heads_shared_stream<2>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+      case 3: return launch_heads_shared_stream<3>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+      case 4: return launch_heads_shared_stream<4>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+      default: return MD_ERR_UNSUPPORTED;
+    }
+  }
+  if (mk <= 4)
+    return launch_heads_shared_gemm<4>(sp, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+  if (mk <= 8)
+    return launch_heads_shared_gemm<8>(sp, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
+  return launch_heads_shared_gemm<16>(sp, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
 }
 
 md_status md_medusa_heads_static(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,

@@ -8,14 +8,15 @@ from __future__ import annotations
 
 import torch
 
-from .binding import (Tree, accept_workspace_bytes, attention_workspace_bytes, heads_workspace_bytes,
-                      medusa_heads, tree_accept, tree_attention, tree_build, tree_commit, workspace)
+from .binding import (Tree, accept_workspace_bytes, attention_workspace_bytes, heads_shared_workspace_bytes,
+                      heads_workspace_bytes, medusa_heads, medusa_heads_shared, tree_accept, tree_attention,
+                      tree_build, tree_commit, workspace)
 from .tree_spec import tree_arrays
 
 
 class MedusaStep:
     def __init__(self, *, B, M, d, V, K, k_per_head, tree_tuples, Hq, Hkv, dh, S_max, mode="greedy",
-                 temperature=0.7, eps=0.09, alpha=0.3, device="cuda", keep_logits=False):
+                 temperature=0.7, eps=0.09, alpha=0.3, device="cuda", keep_logits=False, shared_vocab=False):
         parent, rank = tree_arrays(tree_tuples)
         self.tree = Tree(parent, rank, k_per_head)
         self.B, self.M, self.d, self.V, self.K = B, M, d, V, K
@@ -41,13 +42,16 @@ class MedusaStep:
         self.new_prefix_len = torch.empty((B,), **i32)
         self.next_root = torch.empty((B,), **i32)
         self.next_head_row = torch.empty((B,), **i32)
-        self.ws_heads = workspace(heads_workspace_bytes(M, d, V, K, self.kmax), dev)
+        self.shared_vocab = shared_vocab
+        ws_fn = heads_shared_workspace_bytes if shared_vocab else heads_workspace_bytes
+        self.ws_heads = workspace(ws_fn(M, d, V, K, self.kmax), dev)
         self.ws_attn = workspace(attention_workspace_bytes(B, self.T, Hq, Hkv, dh, S_max), dev)
         self.ws_acc = workspace(accept_workspace_bytes(B, self.T, V), dev)
 
     def heads(self, h, W1, b1, Wv, stream=None):
-        medusa_heads(h, W1, b1, Wv, self.k_per_head, self.topk_ids, self.topk_vals, self.ws_heads,
-                     logits_dbg=self.logits_dbg, stream=stream)
+        fn = medusa_heads_shared if self.shared_vocab else medusa_heads
+        fn(h, W1, b1, Wv, self.k_per_head, self.topk_ids, self.topk_vals, self.ws_heads,
+           logits_dbg=self.logits_dbg, stream=stream)
 
     def build(self, root_token, prefix_len, head_row=None, stream=None):
         tree_build(self.tree, self.topk_ids, root_token, prefix_len, self.tokens, self.parent, self.anc,

@@ -141,6 +141,23 @@ def medusa_heads(h_bits, W1_bits, b1_bits, Wv_bits, k_per_head, kmax=None):
     return ids, vals, logits, z
 
 
+def medusa_heads_shared(h_bits, W1_bits, b1_bits, Wv_bits, k_per_head, kmax=None):
+    """The draft stage with one vocabulary projection shared by every head.
+
+    Source: "Medusa heads versus separate draft model", section "What
+    interviewers probe next": each head normally has its own projection;
+    sharing one saves (K - 1) d V parameters at some cost to acceptance. The
+    residual blocks stay per head; Wv_bits is [d, V].
+    Returns (topk_ids, topk_vals, logits, z_bits).
+    """
+    kmax = max(k_per_head) if kmax is None else kmax
+    z = residual_block(h_bits, W1_bits, b1_bits)
+    K = z.shape[1]
+    logits = vocab_logits(z, np.broadcast_to(Wv_bits, (K,) + Wv_bits.shape))
+    ids, vals = heads_topk(logits, k_per_head, kmax)
+    return ids, vals, logits, z
+
+
 def head_parameter_counts(d: int, V: int, K: int):
     """Parameter counts of the heads as this oracle shapes them.
 

@@ -38,6 +38,7 @@ class Workload:
     eps: float = 0.09
     alpha: float = 0.3
     seed: int = 0
+    shared_vocab: bool = False  # one vocabulary projection for all heads
     extra: dict = field(default_factory=dict)
 
     @property
@@ -59,7 +60,8 @@ class Workload:
         return (s + 63) // 64 * 64
 
     def head_weight_bytes(self) -> int:
-        return 2 * self.K * (self.d * self.d + self.d + self.d * self.V)
+        proj = self.d * self.V * (1 if self.shared_vocab else self.K)
+        return 2 * (self.K * (self.d * self.d + self.d) + proj)
 
 
 TINY = Workload("tiny", B=1, d=256, V=1024, K=4, k_per_head=(4, 3, 2, 2), n_nodes=16,
@@ -76,7 +78,10 @@ BATCHED70B = replace(LLAMA70B, name="llama3-70b-b8", B=8, prefix=(1024, 8192), h
 # so the weights (1.1 GB) exceed L2 while the device footprint stays small.
 PROF_HEADS = replace(LLAMA8B, name="prof-8b-v32000", V=32000)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS)}
+# The same 70B step with one vocabulary projection shared by the four heads.
+LLAMA70B_SHARED = replace(LLAMA70B, name="llama3-70b-shared-proj", shared_vocab=True)
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS, LLAMA70B_SHARED)}
 
 
 def sweep_8b(B: int, tree: str, prefix: int, mode: str = "greedy") -> Workload:

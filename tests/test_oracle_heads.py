@@ -188,3 +188,17 @@ def test_residual_block_column_subset_agrees():
     full = oh.residual_block(h, W1, b1)
     cols = [5, 0, 127, 64]
     assert np.array_equal(oh.residual_block(h, W1, b1, cols=cols), full[:, :, cols])
+
+
+def test_shared_projection_equals_per_head_projections_that_agree():
+    """A shared projection is the per-head form with every Wv_k equal to it."""
+    d, V, K, M = 64, 300, 3, 2
+    h, W1, b1 = (gen.normal_bf16(6, "h", (M, d), 1.0), gen.normal_bf16(6, "W1", (K, d, d), 0.02),
+                 gen.normal_bf16(6, "b1", (K, d), 0.02))
+    Wv = gen.normal_bf16(6, "Wv", (d, V), 0.02)
+    a = oh.medusa_heads_shared(h, W1, b1, Wv, (5, 4, 3))
+    b = oh.medusa_heads(h, W1, b1, np.stack([Wv] * K), (5, 4, 3))
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    # and the saving the page prints: (K - 1) projections of d x V
+    assert (4 - 1) * 8192 * 128256 == 3 * oh.head_parameter_counts(8192, 128256, 4)[1]
