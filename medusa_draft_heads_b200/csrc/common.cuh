@@ -166,6 +166,17 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
+// Element `idx` of a small by-value parameter array without a runtime index into
+// the parameter space (which would copy the whole array to local memory).
+template <int N>
+__device__ __forceinline__ int param_at(const int (&arr)[N], int idx) {
+  int r = 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j)
+    if (j == idx) r = arr[j];
+  return r;
+}
+
 // ---------------------------------------------------------------------------
 // Total order used by every top-k / argmax: larger value first, then lower id.
 // ---------------------------------------------------------------------------

@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kW1Threads) heads_w1_kernel(W1Args a) {
 
   if (col_ok) {
     const uint16_t* wrow = a.W1 + (size_t(k) * d + i0) * d + o;
-    constexpr int U = 4;
+    constexpr int U = M <= 2 ? 8 : 4;      // 16-byte loads in flight per lane
     int r = warp;
     for (; r + (U - 1) * kConsumerWarps < a.rows; r += U * kConsumerWarps) {
       uint4 w[U];
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       }
       float pv = INFINITY;
       int pid = -1;
-      const int kk = a.shared ? a.kph[m % a.kh] : a.kph[k];
+      const int kk = param_at(a.kph, a.shared ? m % a.kh : k);
       float nrv = -INFINITY;
       int nri = INT_MAX;
       for (int r = 0; r < kk; ++r) {
@@ -536,20 +536,42 @@ __global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
   __shared__ int wi[8][kListMax];
   const int mk = blockIdx.x;
   const int k = mk % a.K, m = mk / a.K;
-  const int kk = a.kph[mk % a.kh];
+  const int kk = param_at(a.kph, mk % a.kh);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t base = size_t(mk) * a.nslots * a.kmax;
   const long long run = (long long)(m / a.mrows) * a.K + k;   // (row tile, head) run of (m, k)
   SortedList L;
   L.clear();
+  bool first = true;
   for (int c = threadIdx.x; c < a.nslots; c += 256) {
     if (a.partitioned) {
       const long long u0 = (long long)c * a.units / a.nslots, u1 = (long long)(c + 1) * a.units / a.nslots;
       if (u1 <= run * a.ntiles || u0 >= (run + 1) * a.ntiles) continue;
     }
-    for (int j = 0; j < kk; ++j) {
-      const int id = a.cand_id[base + size_t(c) * a.kmax + j];
-      if (id >= 0) L.push(a.cand_val[base + size_t(c) * a.kmax + j], id);
+    // a slot's list is sorted already: load it whole (independent loads)
+    float lv[kListMax];
+    int li[kListMax];
+#pragma unroll
+    for (int j = 0; j < kListMax; ++j) {
+      const bool use = j < kk;
+      lv[j] = use ? a.cand_val[base + size_t(c) * a.kmax + j] : -INFINITY;
+      li[j] = use ? a.cand_id[base + size_t(c) * a.kmax + j] : -1;
+      if (li[j] < 0) {
+        lv[j] = -INFINITY;
+        li[j] = INT_MAX;
+      }
+    }
+    if (first) {          // the thread's first list becomes its list as it is
+#pragma unroll
+      for (int j = 0; j < kListMax; ++j) {
+        L.v[j] = lv[j];
+        L.i[j] = li[j];
+      }
+      first = false;
+    } else {
+#pragma unroll
+      for (int j = 0; j < kListMax; ++j)
+        if (li[j] != INT_MAX) L.push(lv[j], li[j]);
     }
   }
   float ov;
@@ -561,10 +583,12 @@ __global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
   }
   __syncthreads();
   if (warp == 0) {
-    L.clear();
-    if (lane < 8) {
-      for (int j = 0; j < kk; ++j)
-        if (wi[lane][j] != INT_MAX) L.push(wv[lane][j], wi[lane][j]);
+    // lane l takes warp l's merged list (sorted) as it is
+#pragma unroll
+    for (int j = 0; j < kListMax; ++j) {
+      const bool use = lane < 8 && j < kk;
+      L.v[j] = use ? wv[lane][j] : -INFINITY;
+      L.i[j] = use ? wi[lane][j] : INT_MAX;
     }
     warp_merge(L, kk, lane, ov, oi);
     if (lane < a.kmax) {

@@ -152,9 +152,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + size_t(slot) * kStageBytes;
           mbar_arrive_expect_tx(fb, kStageBytes);
           tma_load_3d(smem_u32(st), &amap, s * kBK, mt * kBM, a.a_shared ? 0 : k, fb);
+          // A weight strip is read once per row tile: stream it evict-first only when
+          // there is a single row tile, otherwise keep it in L2 for the other tiles.
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_load_3d_hint(smem_u32(st + kABytes + j * kBBox), &bmap, nt * kBN + j * 64, s * kBK, k, fb, pol);
+          for (int j = 0; j < 4; ++j) {
+            if (a.mtiles == 1)
+              tma_load_3d_hint(smem_u32(st + kABytes + j * kBBox), &bmap, nt * kBN + j * 64, s * kBK, k, fb, pol);
+            else
+              tma_load_3d(smem_u32(st + kABytes + j * kBBox), &bmap, nt * kBN + j * 64, s * kBK, k, fb);
+          }
         }
       }
       for (int j = (it > kStages ? it - kStages : 0); j < it; ++j) {
@@ -249,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         if (k != cur_k) {         // a new (row tile, head) run starts: fresh lists
-          L.kk = a.kh > 0 ? a.kph[m % a.kh] : a.kph[k];
+          L.kk = param_at(a.kph, a.kh > 0 ? m % a.kh : k);
           L.reset();
           cur_k = k;
         }

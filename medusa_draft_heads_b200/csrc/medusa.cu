@@ -406,7 +406,7 @@ AcceptPlan accept_plan(int B, int T, int V) {
   AcceptPlan p;
   const int rows = B * T;
   const int max_chunks = (V + 1023) / 1024;
-  int n = (2 * num_sms() + rows - 1) / rows;
+  int n = (4 * num_sms() + rows - 1) / rows;      // ~4 CTAs per SM: enough loads in flight
   n = std::max(1, std::min(n, max_chunks));
   int len = (V + n - 1) / n;
   len = (len + 1023) / 1024 * 1024;

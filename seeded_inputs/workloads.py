@@ -77,11 +77,14 @@ BATCHED70B = replace(LLAMA70B, name="llama3-70b-b8", B=8, prefix=(1024, 8192), h
 # Profiling case for the heads kernels: 8B-shaped with a 32000-token vocabulary,
 # so the weights (1.1 GB) exceed L2 while the device footprint stays small.
 PROF_HEADS = replace(LLAMA8B, name="prof-8b-v32000", V=32000)
+# Profiling case for the tensor-core heads: the same weights on 8 x 65 = 520 rows.
+PROF_GEMM = replace(PROF_HEADS, name="prof-8b-v32000-b8", B=8, heads_rows="BT", prefix=(1024, 8192))
 
 # The same 70B step with one vocabulary projection shared by the four heads.
 LLAMA70B_SHARED = replace(LLAMA70B, name="llama3-70b-shared-proj", shared_vocab=True)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS, LLAMA70B_SHARED)}
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS, PROF_GEMM,
+                                 LLAMA70B_SHARED)}
 
 
 def sweep_8b(B: int, tree: str, prefix: int, mode: str = "greedy") -> Workload:
