@@ -452,9 +452,9 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 // Phase 3: merge candidate lists into each head's top-k.
 // grid (M * K), 256 threads. The candidates of (m, k) are `nslots` lists of
 // up to kmax entries. In "partitioned" mode slot c is CTA c of the kernel that
-// produced them: that kernel split `units` work units, ordered (row tile of
-// `mrows` rows, head, column tile of `ntiles`), into contiguous CTA ranges, and
-// only CTAs whose range touches the (row tile of m, head k) run wrote a list. Each
+// produced them (the CTAs that worked on row m): that kernel split `units`
+// work units, ordered (head, column tile of `ntiles`), into contiguous CTA
+// ranges, and only CTAs whose range touches head k wrote a list. Each
 // thread gathers its slots into a sorted register list; each warp then merges
 // its 32 lists by k rounds of a shuffle arg-max over the list heads (the
 // winning lane shifts its list), and warp 0 merges the 8 warp lists the same way.
@@ -465,7 +465,7 @@ struct MergeArgs {
   int32_t* topk_ids;   // [M, K, kmax]
   float* topk_vals;
   int K, kmax, nslots;
-  int partitioned, units, ntiles, mrows;   // producer partition (partitioned == 1)
+  int partitioned, units, ntiles;   // producer partition (partitioned == 1)
   int kh;              // heads for the top-k size: row mk uses kph[mk % kh]
   int kph[MD_MAX_K];
 };
@@ -535,18 +535,17 @@ __global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
   __shared__ float wv[8][kListMax];
   __shared__ int wi[8][kListMax];
   const int mk = blockIdx.x;
-  const int k = mk % a.K, m = mk / a.K;
+  const int k = mk % a.K;
   const int kk = param_at(a.kph, mk % a.kh);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t base = size_t(mk) * a.nslots * a.kmax;
-  const long long run = (long long)(m / a.mrows) * a.K + k;   // (row tile, head) run of (m, k)
   SortedList L;
   L.clear();
   bool first = true;
   for (int c = threadIdx.x; c < a.nslots; c += 256) {
     if (a.partitioned) {
       const long long u0 = (long long)c * a.units / a.nslots, u1 = (long long)(c + 1) * a.units / a.nslots;
-      if (u1 <= run * a.ntiles || u0 >= (run + 1) * a.ntiles) continue;
+      if (u1 <= (long long)k * a.ntiles || u0 >= (long long)(k + 1) * a.ntiles) continue;
     }
     // a slot's list is sorted already: load it whole (independent loads)
     float lv[kListMax];

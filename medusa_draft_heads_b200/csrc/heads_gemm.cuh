@@ -18,12 +18,18 @@
 // accumulators in tensor memory (512 columns), warps 2..5 drain the other
 // accumulator through tcgen05.ld (one TMEM lane = one row per thread).
 //
-// Tiles are ordered (row tile, head, column tile) and CTA c takes the
-// contiguous range [c*U/G, (c+1)*U/G), so the CTAs working on different row
-// tiles walk the same weight columns at the same time (the weight strip is
-// read from HBM once and then from L2), and in phase 2 each row keeps one
-// running top-k across the CTA's column tiles: after the first tiles nearly
-// every logit is rejected by one compare against the current k-th best.
+// Work split: the grid is mtiles groups of per_mt CTAs, group g takes row
+// tile g, and CTA j of every group takes the same contiguous range
+// [j*U/per_mt, (j+1)*U/per_mt) of the U = K * ntiles (head, column tile)
+// units. The CTAs with the same j therefore walk the same weight strips in
+// step: a strip comes from HBM once and from L2 for the other row tiles, and
+// the strips in flight at any moment (per_mt of them) fit in L2. (Contiguous
+// ranges over all tiles would put the CTAs of different row tiles on
+// different strips at any one time; with mtiles x per_mt strips in flight the
+// reuse distance exceeds L2 and every row tile re-reads its strips from HBM.)
+// In phase 2 each row keeps one running top-k across the CTA's column tiles:
+// after the first tiles nearly every logit is rejected by one compare against
+// the current k-th best.
 #pragma once
 
 #include "common.cuh"
@@ -46,12 +52,14 @@ enum { EPI_SILU = 0, EPI_TOPK = 1 };
 
 struct Args {
   int M, d, N, K;                 // rows, reduction length, output columns, heads
-  int mtiles, ntiles, tiles;      // tiles = mtiles * K * ntiles, ordered (mtile, head, ntile)
+  int ntiles;                     // column tiles per head
+  int per_mt;                     // CTAs (pairs) per row tile (pair) group
+  int groups;                     // CTA-pair kernel: row-pair groups (grid = 2 x groups x per_mt)
   int a_shared;                   // A is one matrix for every head (phase 1: h)
   const uint16_t* h;              // [M, d]      phase 1 residual
   const uint16_t* b1;             // [K, d]      phase 1 bias
   uint16_t* zg;                   // [K, M, d]   phase 1 output
-  float* cand_val;                // [M, K, gridDim.x, kmax]  phase 2: one list per (row, head, CTA)
+  float* cand_val;                // [M, K, per_mt, kmax]  phase 2: one list per (row, head, CTA of the row tile)
   int* cand_id;
   float* logits_dbg;              // [M, K, N] or null
   int kmax;
@@ -90,6 +98,53 @@ struct SmemList {
   }
 };
 
+// Phase-1 epilogue for 32 columns o0.. of row m, head k: z = bf16(h + SiLU(acc + b1)).
+__device__ __forceinline__ void silu_residual_store(const Args& a, int m, int k, int o0, const float (&v)[32]) {
+  const uint4* hp = reinterpret_cast<const uint4*>(a.h + size_t(m) * a.d + o0);
+  const uint4* bp = reinterpret_cast<const uint4*>(a.b1 + size_t(k) * a.d + o0);
+  uint4* zp = reinterpret_cast<uint4*>(a.zg + (a.zg_mk ? size_t(m) * a.K + k : size_t(k) * a.M + m) * a.d + o0);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint4 hv = hp[g], bv = __ldg(bp + g);
+    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+    uint32_t zw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float u0 = v[g * 8 + 2 * e] + bf16lo(bw[e]);
+      const float u1 = v[g * 8 + 2 * e + 1] + bf16hi(bw[e]);
+      const uint16_t z0 = f32_to_bf16_rne(bf16lo(hw[e]) + u0 / (1.0f + expf(-u0)));
+      const uint16_t z1 = f32_to_bf16_rne(bf16hi(hw[e]) + u1 / (1.0f + expf(-u1)));
+      zw[e] = uint32_t(z0) | (uint32_t(z1) << 16);
+    }
+    zp[g] = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+  }
+}
+
+// Phase-2 epilogue for 32 logits of row m, head k, columns c0..: fold them
+// into the running top-k (and copy them out when the debug logits are kept).
+__device__ __forceinline__ void topk_tile_columns(const Args& a, SmemList& L, int m, int k, int c0,
+                                                  const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (c0 + j < a.N && better(v[j], c0 + j, L.tv, L.ti)) L.insert(v[j], c0 + j);
+  if (a.logits_dbg) {
+    float* lp = a.logits_dbg + (size_t(m) * a.K + k) * a.N + c0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      if (c0 + j < a.N) *reinterpret_cast<float4*>(lp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  }
+}
+
+// Write a running list to candidate slot `slot` of (row m, head k).
+__device__ __forceinline__ void flush_list(const Args& a, const SmemList& L, int m, int k, int slot) {
+  const size_t cb = ((size_t(m) * a.K + k) * a.per_mt + slot) * a.kmax;
+  for (int j = 0; j < L.kk; ++j) {
+    a.cand_val[cb + j] = L.v[j * 128];
+    a.cand_id[cb + j] = L.i[j * 128] == INT_MAX ? -1 : L.i[j * 128];
+  }
+}
+
 template <int EPI, int KK>
 __global__ void __launch_bounds__(kThreads, 1)
     heads_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, Args a) {
@@ -105,8 +160,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = a.d / kBK;
-  const int t_begin = int((long long)blockIdx.x * a.tiles / gridDim.x);
-  const int t_end = int((long long)(blockIdx.x + 1) * a.tiles / gridDim.x);
+  const int mt = blockIdx.x / a.per_mt, cj = blockIdx.x % a.per_mt;
+  const int units = a.K * a.ntiles;
+  const int t_begin = int((long long)cj * units / a.per_mt);
+  const int t_end = int((long long)(cj + 1) * units / a.per_mt);
   pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
@@ -139,8 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = t_begin; tile < t_end && ok; ++tile) {
-        const int nt = tile % a.ntiles, r = tile / a.ntiles;
-        const int k = r % a.K, mt = r / a.K;
+        const int nt = tile % a.ntiles, k = tile / a.ntiles;
         for (int s = 0; s < nk; ++s, ++it) {
           const int slot = it % kStages;
           if (it >= kStages && !mbar_wait(smem_u32(&empty[slot]), ((it / kStages) - 1) & 1)) {
@@ -156,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // there is a single row tile, otherwise keep it in L2 for the other tiles.
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            if (a.mtiles == 1)
+            if (gridDim.x == a.per_mt)
               tma_load_3d_hint(smem_u32(st + kABytes + j * kBBox), &bmap, nt * kBN + j * 64, s * kBK, k, fb, pol);
             else
               tma_load_3d(smem_u32(st + kABytes + j * kBBox), &bmap, nt * kBN + j * 64, s * kBK, k, fb);
@@ -214,8 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lt = 0;
     int cur_k = -1;
     for (int tile = t_begin; tile < t_end; ++tile, ++lt) {
-      const int nt = tile % a.ntiles, r = tile / a.ntiles;
-      const int k = r % a.K, mt = r / a.K;
+      const int nt = tile % a.ntiles, k = tile / a.ntiles;
       const int buf = lt & 1;
       if (!mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1)) {
         set_status(MD_DEV_TIMEOUT);
@@ -230,31 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
           tmem_ld32(tbase + c, v);
           const int o0 = nt * kBN + c;
-          if (live && o0 < a.d) {
-            const uint4* hp = reinterpret_cast<const uint4*>(a.h + size_t(m) * a.d + o0);
-            const uint4* bp = reinterpret_cast<const uint4*>(a.b1 + size_t(k) * a.d + o0);
-            uint4* zp = reinterpret_cast<uint4*>(
-                a.zg + (a.zg_mk ? size_t(m) * a.K + k : size_t(k) * a.M + m) * a.d + o0);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint4 hv = hp[g], bv = __ldg(bp + g);
-              const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-              const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-              uint32_t zw[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float u0 = v[g * 8 + 2 * e] + bf16lo(bw[e]);
-                const float u1 = v[g * 8 + 2 * e + 1] + bf16hi(bw[e]);
-                const uint16_t z0 = f32_to_bf16_rne(bf16lo(hw[e]) + u0 / (1.0f + expf(-u0)));
-                const uint16_t z1 = f32_to_bf16_rne(bf16hi(hw[e]) + u1 / (1.0f + expf(-u1)));
-                zw[e] = uint32_t(z0) | (uint32_t(z1) << 16);
-              }
-              zp[g] = make_uint4(zw[0], zw[1], zw[2], zw[3]);
-            }
-          }
+          if (live && o0 < a.d) silu_residual_store(a, m, k, o0, v);
         }
       } else {
-        if (k != cur_k) {         // a new (row tile, head) run starts: fresh lists
+        if (k != cur_k) {         // a new head starts: fresh lists
           L.kk = param_at(a.kph, a.kh > 0 ? m % a.kh : k);
           L.reset();
           cur_k = k;
@@ -263,28 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
           tmem_ld32(tbase + c, v);
           const int c0 = nt * kBN + c;
-          if (live) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < a.N && better(v[j], c0 + j, L.tv, L.ti)) L.insert(v[j], c0 + j);
-            if (a.logits_dbg) {
-              float* lp = a.logits_dbg + (size_t(m) * a.K + k) * a.N + c0;
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                if (c0 + j < a.N) *reinterpret_cast<float4*>(lp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-            }
-          }
+          if (live) topk_tile_columns(a, L, m, k, c0, v);
         }
-        // flush at the end of a (row tile, head) run
+        // flush at the end of the CTA's run of this head
         const bool last = tile + 1 == t_end || (tile + 1) / a.ntiles != tile / a.ntiles;
         if (last) {
-          if (live) {
-            const size_t cb = ((size_t(m) * a.K + k) * gridDim.x + blockIdx.x) * a.kmax;
-            for (int j = 0; j < L.kk; ++j) {
-              a.cand_val[cb + j] = L.v[j * 128];
-              a.cand_id[cb + j] = L.i[j * 128] == INT_MAX ? -1 : L.i[j * 128];
-            }
-          }
+          if (live) flush_list(a, L, m, k, cj);
           cur_k = -1;
         }
       }

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "heads.cuh"
 #include "heads_gemm.cuh"
+#include "heads_gemm2.cuh"
 #include "tree_build.cuh"
 #include "attention.cuh"
 #include "attention_tc.cuh"
@@ -163,18 +164,57 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = pl.K; ma.kmax = pl.kmax; ma.nslots = pl.grid;
-  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.mrows = 1 << 30; ma.kh = pl.K;
+  ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.kh = pl.K;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
   return launch_pdl(heads_merge_kernel, dim3(pl.M * pl.K), dim3(256), 0, st, ma);
 }
 
-// Workspace of the tensor-core path (M > 8): z [K, M, d] bf16 and the
-// per-tile candidates [M, K, ceil(V/256), kmax].
+// Workspace of the tensor-core path: z [K, M, d] bf16 and the candidates
+// [M, K, per_mt2, kmax] (one list per row, head and CTA / CTA pair of the
+// row's tile). More than one 128-row tile: CTA pairs (256-row tiles).
 struct GemmPlan {
   int mtiles, ntiles1, ntiles2;
-  int grid1, grid2;   // CTAs of the two GEMMs (one candidate list per row, head and CTA in phase 2)
+  bool pair;              // CTA-pair kernel (M > 128)
+  int groups;             // row tiles (single CTAs) or row-tile pairs (pairs)
+  int cluster;            // pair kernel: CTAs per cluster (2 * groups when <= 8, else 2)
+  int per_mt1, per_mt2;   // CTAs (pairs) per group of the two GEMMs
+  int grid1, grid2;
   size_t off_z, off_cval, off_cid, bytes;
 };
+
+// Clusters of `cs` CTAs of the pair kernel that can be resident at once
+// (0 when such a cluster cannot be placed).
+int pair_max_clusters(int cs) {
+  static std::mutex mu;
+  static int cache[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[cs] >= 0) return cache[cs];
+  auto kern = md::gemm::heads_gemm_pair_kernel<md::gemm::EPI_TOPK, 16>;
+  int n = 0;
+  if (set_smem(kern, md::gemm::kSmemP) == MD_OK) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs * 64);
+    cfg.blockDim = dim3(md::gemm::kThreads);
+    cfg.dynamicSmemBytes = md::gemm::kSmemP;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  cache[cs] = n;
+  return n;
+}
+
+// CTAs (pairs) per group: as many as can be resident side by side with the
+// other groups, at most one per (head, column tile) unit.
+inline int gemm_per_mt(int slots, int groups, int units) { return std::max(1, std::min(slots / groups, units)); }
 
 GemmPlan gemm_plan(int M, int d, int V, int K, int kmax) {
   using md::heads::align256;
@@ -182,12 +222,27 @@ GemmPlan gemm_plan(int M, int d, int V, int K, int kmax) {
   p.mtiles = (M + md::gemm::kBM - 1) / md::gemm::kBM;
   p.ntiles1 = (d + md::gemm::kBN - 1) / md::gemm::kBN;
   p.ntiles2 = (V + md::gemm::kBN - 1) / md::gemm::kBN;
-  p.grid1 = std::min(num_sms(), K * p.ntiles1 * p.mtiles);
-  p.grid2 = std::min(num_sms(), K * p.ntiles2 * p.mtiles);
+  p.pair = p.mtiles > 1;
+  p.groups = p.pair ? (p.mtiles + 1) / 2 : p.mtiles;
+  int slots = num_sms();
+  p.cluster = 0;
+  if (p.pair) {
+    p.cluster = 2;
+    int nc = pair_max_clusters(p.cluster);
+    if (nc <= 0 && p.cluster > 2) {
+      p.cluster = 2;
+      nc = pair_max_clusters(2);
+    }
+    slots = std::max(1, nc) * p.cluster / 2;   // resident pairs
+  }
+  p.per_mt1 = gemm_per_mt(slots, p.groups, K * p.ntiles1);
+  p.per_mt2 = gemm_per_mt(slots, p.groups, K * p.ntiles2);
+  p.grid1 = p.groups * p.per_mt1 * (p.pair ? 2 : 1);
+  p.grid2 = p.groups * p.per_mt2 * (p.pair ? 2 : 1);
   size_t o = 0;
   p.off_z = o;    o = align256(o + size_t(K) * M * d * 2);
-  p.off_cval = o; o = align256(o + size_t(M) * K * p.grid2 * kmax * 4);
-  p.off_cid = o;  o = align256(o + size_t(M) * K * p.grid2 * kmax * 4);
+  p.off_cval = o; o = align256(o + size_t(M) * K * p.per_mt2 * kmax * 4);
+  p.off_cid = o;  o = align256(o + size_t(M) * K * p.per_mt2 * kmax * 4);
   p.bytes = o;
   return p;
 }
@@ -208,21 +263,34 @@ md_status make_map_3d_sw128(CUtensorMap* map, const void* base, uint64_t n0, uin
 }
 
 template <int EPI, int KK>
-md_status launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const md::gemm::Args& ga, bool pdl,
-                      cudaStream_t st) {
+md_status launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const md::gemm::Args& ga, int grid,
+                      int cluster, bool pdl, cudaStream_t st) {
   md_status s;
-  auto kern = md::gemm::heads_gemm_kernel<EPI, KK>;
-  if ((s = set_smem(kern, md::gemm::kSmem)) != MD_OK) return s;
+  const bool pair = cluster > 0;
+  auto kern = pair ? md::gemm::heads_gemm_pair_kernel<EPI, KK> : md::gemm::heads_gemm_kernel<EPI, KK>;
+  const int smem = pair ? md::gemm::kSmemP : md::gemm::kSmem;
+  if ((s = set_smem(kern, smem)) != MD_OK) return s;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min(num_sms(), ga.tiles));
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(md::gemm::kThreads);
-  cfg.dynamicSmemBytes = md::gemm::kSmem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pair) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   return cuda_ok(cudaLaunchKernelEx(&cfg, kern, amap, bmap, ga));
 }
 
@@ -234,7 +302,7 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   const GemmPlan pl = gemm_plan(M, d, V, K, kmax);
   md_status s;
   Args ga = {};
-  ga.M = M; ga.d = d; ga.K = K; ga.mtiles = pl.mtiles; ga.kmax = kmax;
+  ga.M = M; ga.d = d; ga.K = K; ga.kmax = kmax;
   ga.h = h; ga.b1 = b1;
   ga.zg = reinterpret_cast<uint16_t*>(ws + pl.off_z);
   ga.cand_val = reinterpret_cast<float*>(ws + pl.off_cval);
@@ -246,21 +314,21 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   CUtensorMap amap, bmap;
   if ((s = make_map_3d_sw128(&amap, h, d, M, 1, kBK, kBM)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&bmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
-  ga.N = d; ga.ntiles = pl.ntiles1; ga.tiles = K * pl.ntiles1 * pl.mtiles; ga.a_shared = 1;
-  if ((s = launch_gemm<EPI_SILU, KK>(amap, bmap, ga, false, st)) != MD_OK) return s;
+  ga.N = d; ga.ntiles = pl.ntiles1; ga.per_mt = pl.per_mt1; ga.groups = pl.groups; ga.a_shared = 1;
+  if ((s = launch_gemm<EPI_SILU, KK>(amap, bmap, ga, pl.grid1, pl.cluster, false, st)) != MD_OK) return s;
 
   // phase 2: logits tile = z_k Wv_k, per-row top-k of every 256-column tile
   if ((s = make_map_3d_sw128(&amap, ga.zg, d, M, K, kBK, kBM)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&bmap, Wv, V, d, K, 64, kBK)) != MD_OK) return s;
-  ga.N = V; ga.ntiles = pl.ntiles2; ga.tiles = K * pl.ntiles2 * pl.mtiles; ga.a_shared = 0;
-  if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, true, st)) != MD_OK) return s;
+  ga.N = V; ga.ntiles = pl.ntiles2; ga.per_mt = pl.per_mt2; ga.groups = pl.groups; ga.a_shared = 0;
+  if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, pl.grid2, pl.cluster, true, st)) != MD_OK) return s;
 
   // phase 3: merge the tiles' candidates
   md::heads::MergeArgs ma;
   ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
-  ma.K = K; ma.kmax = kmax; ma.nslots = pl.grid2;
-  ma.partitioned = 1; ma.units = K * pl.ntiles2 * pl.mtiles; ma.ntiles = pl.ntiles2; ma.mrows = kBM; ma.kh = K;
+  ma.K = K; ma.kmax = kmax; ma.nslots = pl.per_mt2;
+  ma.partitioned = 1; ma.units = K * pl.ntiles2; ma.ntiles = pl.ntiles2; ma.kh = K;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
   return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
 }
@@ -344,7 +412,7 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   ma.cand_val = va.cand_val; ma.cand_id = va.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = 1; ma.kmax = p2.kmax; ma.nslots = p2.grid;
-  ma.partitioned = 1; ma.units = p2.units; ma.ntiles = p2.ntiles; ma.mrows = 1 << 30; ma.kh = p1.K;
+  ma.partitioned = 1; ma.units = p2.units; ma.ntiles = p2.ntiles; ma.kh = p1.K;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
   return launch_pdl(heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
 }
@@ -368,20 +436,20 @@ md_status launch_heads_shared_gemm(const SharedPlan& sp, int M, int d, int V, in
   CUtensorMap amap, bmap;
   if ((s = make_map_3d_sw128(&amap, h, d, M, 1, kBK, kBM)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&bmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
-  ga.M = M; ga.K = K; ga.N = d; ga.mtiles = sp.g1.mtiles; ga.ntiles = sp.g1.ntiles1;
-  ga.tiles = K * sp.g1.ntiles1 * sp.g1.mtiles; ga.a_shared = 1; ga.zg_mk = 1; ga.kh = 0;
-  if ((s = launch_gemm<EPI_SILU, KK>(amap, bmap, ga, false, st)) != MD_OK) return s;
+  ga.M = M; ga.K = K; ga.N = d; ga.ntiles = sp.g1.ntiles1; ga.per_mt = sp.g1.per_mt1; ga.groups = sp.g1.groups;
+  ga.a_shared = 1; ga.zg_mk = 1; ga.kh = 0;
+  if ((s = launch_gemm<EPI_SILU, KK>(amap, bmap, ga, sp.g1.grid1, sp.g1.cluster, false, st)) != MD_OK) return s;
   // phase 2: the M*K rows against the one projection
   if ((s = make_map_3d_sw128(&amap, ga.zg, d, MK, 1, kBK, kBM)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&bmap, Wv, V, d, 1, 64, kBK)) != MD_OK) return s;
-  ga.M = MK; ga.K = 1; ga.N = V; ga.mtiles = sp.g2.mtiles; ga.ntiles = sp.g2.ntiles2;
-  ga.tiles = sp.g2.ntiles2 * sp.g2.mtiles; ga.a_shared = 1; ga.zg_mk = 0; ga.kh = K;
-  if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, true, st)) != MD_OK) return s;
+  ga.M = MK; ga.K = 1; ga.N = V; ga.ntiles = sp.g2.ntiles2; ga.per_mt = sp.g2.per_mt2; ga.groups = sp.g2.groups;
+  ga.a_shared = 1; ga.zg_mk = 0; ga.kh = K;
+  if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, sp.g2.grid2, sp.g2.cluster, true, st)) != MD_OK) return s;
   md::heads::MergeArgs ma;
   ma.cand_val = ga.cand_val; ma.cand_id = ga.cand_id;
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
-  ma.K = 1; ma.kmax = kmax; ma.nslots = sp.g2.grid2;
-  ma.partitioned = 1; ma.units = sp.g2.ntiles2 * sp.g2.mtiles; ma.ntiles = sp.g2.ntiles2; ma.mrows = kBM; ma.kh = K;
+  ma.K = 1; ma.kmax = kmax; ma.nslots = sp.g2.per_mt2;
+  ma.partitioned = 1; ma.units = sp.g2.ntiles2; ma.ntiles = sp.g2.ntiles2; ma.kh = K;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
   return launch_pdl(md::heads::heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
 }

@@ -96,7 +96,7 @@ def test_heads_reject_bad_arguments():
                         vals, ws)
 
 
-# ----------------------------- tensor-core path (M > 8) -----------------------------
+# ------------- tensor-core path (M > 4; CTA pairs once M > 128 rows) -------------
 
 @pytest.mark.parametrize("M,d,V,kph", [(9, 256, 1024, (4, 3, 2, 2)), (40, 320, 1000, (10, 10, 10, 10)),
                                        (130, 512, 2056, (16, 1, 7, 3)), (520, 256, 4096, (10, 10, 10, 10))])
@@ -112,7 +112,8 @@ def test_tensor_core_heads_match_oracle(M, d, V, kph):
             check_topk_row(ids[m, k], vals[m, k], rlog[m, k], kk)
 
 
-@pytest.mark.parametrize("M,d,V,kph", [(17, 128, 1024, (16, 10, 1, 5)), (200, 64, 776, (3, 16, 2, 9))])
+@pytest.mark.parametrize("M,d,V,kph", [(17, 128, 1024, (16, 10, 1, 5)), (200, 64, 776, (3, 16, 2, 9)),
+                                       (300, 128, 520, (8, 2))])
 def test_tensor_core_topk_bit_exact_on_integer_logits(M, d, V, kph):
     h, W1, b1, Wv = _integer_heads(M * 3 + d, M, d, V, len(kph))
     ids, vals, logits = _run(h, W1, b1, Wv, kph)
