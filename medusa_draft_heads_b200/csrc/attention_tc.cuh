@@ -11,22 +11,26 @@
 // loaded by one 3-D TMA box straight out of q[B, T, Hq, dh]. The CTA walks its
 // share of 128-key chunks:
 //
-//   warp 0     TMA: the Q tile once, then K and V chunks into two 2-deep rings
+//   warp 0     TMA: the Q tile once, then K and V chunks into two 3-deep rings
 //              (a K slot frees when its S is done, a V slot when its P V is)
-//   warp 1     one thread issues S_c = Q K_c^T into TMEM (double-buffered, two
+//   warp 1     one thread issues S_c = Q K_c^T into TMEM (three buffers, three
 //              chunks ahead) and O += P_c V_c into one TMEM accumulator that
-//              lives across chunks
+//              lives across chunks, with P_c read from TMEM
 //   warps 2-9  two warps per TMEM lane quarter, each taking half of the keys of
 //              a row (row maxima are exchanged through shared memory): read
-//              S_c from TMEM, apply the scale
-//              and -- only in chunks that reach the tree slots -- the tree
-//              mask (a key at slot >= P_b is tree node slot - P_b, visible iff
-//              it is an ancestor-or-self), then P_c = exp2(S - m) against a
-//              running row maximum m, split into bf16 hi + lo parts in
-//              swizzled shared memory (P V runs as P_hi V + P_lo V, keeping
-//              ~16 significant bits of each weight). m only moves when a chunk
-//              exceeds it by more than 2^8; O and the row sum are then rescaled
-//              in place.
+//              S_c from TMEM, apply the scale and -- only in chunks that reach
+//              the tree slots -- the tree mask (a key at slot >= P_b is tree
+//              node slot - P_b, visible iff it is an ancestor-or-self), then
+//              P_c = exp2(S - m) against a running row maximum m, split into
+//              bf16 hi + lo parts (P V runs as P_hi V + P_lo V, keeping ~16
+//              significant bits of each weight) and written back over S_c's
+//              own TMEM columns. m only moves when a chunk exceeds it by more
+//              than 2^8; O and the row sum are then rescaled in place.
+//
+// Because P_c lives in S_c's buffer, the softmax of chunk c + 1 never waits for
+// P_c V_c (only a rescale of O does), and with three buffers S_{c+1}, S_{c+2}
+// are computed while the softmax works on c: the softmax warps and the tensor
+// pipe work on different chunks at the same time.
 //
 // Each CTA writes its split's (m, sum, unnormalised O) per row; the last CTA of
 // a (request, KV head, row tile) to finish combines the splits in split order
@@ -46,6 +50,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;   // lazy rescale threshold (factor 256)
 constexpr int kMaxSplits = 16;
 
+constexpr int kStages = 3;      // K / V ring depth
+constexpr int kSBufs = 3;       // S / P buffers in TMEM (3 x 128 columns + O)
+
 template <int DH>
 struct Cfg {
   static constexpr int KB = DH / 64;                          // 64-element blocks of the head dim
@@ -53,8 +60,7 @@ struct Cfg {
   static constexpr uint32_t kKBytes = KB * kBN * 128;         // K chunk, K-major SW128
   static constexpr uint32_t kVBytes = KB * kBN * 128;         // V chunk, N(dh)-major SW128
   static constexpr uint32_t kStage = kKBytes + kVBytes;
-  static constexpr uint32_t kPBytes = 2 * kBM * 128;          // P tile: 128 rows x 128 keys bf16
-  static constexpr int kSmem = kQBytes + 2 * kStage + 2 * kPBytes + 1024 + 256 + 1024;  // P hi/lo, maxima
+  static constexpr int kSmem = kQBytes + kStages * kStage + 1024 + 256 + 1024;  // + barriers, maxima
 };
 
 struct Args {
@@ -67,12 +73,26 @@ struct Args {
   float scale_log2;
 };
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// 2^x on the special-function unit; results below 2^-126 flush to zero (a
+// weight that small is far below the bf16 hi/lo resolution of the row's sum).
+__device__ __forceinline__ float exp2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__device__ __forceinline__ bool tree_visible(const TreeParams& tp, int t, int node) {
-  return (tp.anc[t][node >> 5] >> (node & 31)) & 1u;
+// Visibility of the 64 keys n0 .. n0 + 63 (n = slot - P: negative n is a
+// prefix key, always visible; tree node n is visible iff it is an ancestor-or-
+// self of the row's token) as bit j, from the row's 128-bit ancestor set
+// (lo = nodes 0..63, hi = nodes 64..127; bits of nodes >= T are zero).
+__device__ __forceinline__ uint64_t visible_bits(uint64_t lo, uint64_t hi, int n0) {
+  if (n0 <= -64) return ~0ull;
+  if (n0 >= 128) return 0ull;
+  if (n0 < 0) return (lo << (-n0)) | ((1ull << (-n0)) - 1ull);
+  if (n0 == 0) return lo;
+  if (n0 < 64) return (lo >> n0) | (hi << (64 - n0));
+  if (n0 == 64) return hi;
+  return hi >> (n0 - 64);
 }
 
 template <int DH>
@@ -83,22 +103,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::kQBytes;                     // 2 stages of (K, V)
-  uint8_t* sP = sKV + 2 * C::kStage;                    // P hi
-  uint8_t* sPl = sP + C::kPBytes;                       // P lo
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sPl + C::kPBytes);
-  uint64_t* q_full = bars;            // 1
-  uint64_t* k_full = bars + 1;        // 2
-  uint64_t* k_empty = bars + 3;       // 2
-  uint64_t* v_full = bars + 5;        // 2
-  uint64_t* v_empty = bars + 7;       // 2
-  uint64_t* s_full = bars + 9;        // 2
-  uint64_t* s_empty = bars + 11;      // 2
-  uint64_t* p_full = bars + 13;       // 1
-  uint64_t* o_full = bars + 14;       // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
-  int* last_flag = reinterpret_cast<int*>(bars + 16);
-  float* xmax = reinterpret_cast<float*>(bars + 17);    // [2 halves][128 rows] chunk maxima
+  uint8_t* sKV = smem + C::kQBytes;                     // kStages stages of (K, V)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kStages * C::kStage);
+  uint64_t* q_full = bars;                      // 1
+  uint64_t* k_full = q_full + 1;                // kStages
+  uint64_t* k_empty = k_full + kStages;         // kStages
+  uint64_t* v_full = k_empty + kStages;         // kStages
+  uint64_t* v_empty = v_full + kStages;         // kStages
+  uint64_t* s_full = v_empty + kStages;         // kSBufs
+  uint64_t* p_full = s_full + kSBufs;           // kSBufs
+  uint64_t* o_full = p_full + kSBufs;           // 2: P_c V_c commits to o_full[c & 1]
+  uint64_t* o_last = o_full + 2;                // 1: every P V done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + 1);
+  int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
+  float* xmax = reinterpret_cast<float*>(bars + 32);    // [2 halves][128 rows] chunk maxima
 
   const int split = blockIdx.x, rt = blockIdx.y % a.rtiles, hk = blockIdx.y / a.rtiles, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,16 +134,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_empty[i]), kSoftWarps);
     }
-    mbar_init(smem_u32(p_full), kSoftWarps);
-    mbar_init(smem_u32(o_full), 1);
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&p_full[i]), kSoftWarps);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&o_full[i]), 1);
+    mbar_init(smem_u32(o_last), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -136,8 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;                 // S_c at columns [128*(c&1), +128)
-  const uint32_t tO = tmem + 2 * kBN;       // O at columns [256, 256 + DH)
+  // S_c at columns [128*(c%3), +128); P_c overwrites them: hi parts in the
+  // first 64 columns, lo parts in the last 64 (two bf16 keys per column)
+  const uint32_t tS = tmem;
+  const uint32_t tO = tmem + kSBufs * kBN;  // O at columns [384, 384 + DH)
   const int kvrow = b * a.Hkv + hk;
   const int tpt = kBM / a.G;                // tree tokens per query tile
 
@@ -154,25 +176,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(smem_u32(sQ + kb * kBM * 128), &qmap, kb * 64, hk * a.G, b * T + rt * tpt, qb);
       bool ok = true;
       for (int c = 0; c < nch && ok; ++c) {
-        const int st = c & 1;
+        const int st = c % kStages, ph = ((c / kStages) - 1) & 1;
         const int key0 = (c_begin + c) * kBN;
         uint8_t* sk = sKV + st * C::kStage;
         uint8_t* sv = sk + C::kKBytes;
-        if (c >= 2 && !mbar_wait(smem_u32(&k_empty[st]), ((c >> 1) - 1) & 1)) { ok = false; break; }
+        if (c >= kStages && !mbar_wait(smem_u32(&k_empty[st]), ph)) { ok = false; break; }
         const uint32_t kb_ = smem_u32(&k_full[st]);
         mbar_arrive_expect_tx(kb_, C::kKBytes);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(smem_u32(sk + kb * kBN * 128), &kmap, kb * 64, key0, kvrow, kb_);
-        if (c >= 2 && !mbar_wait(smem_u32(&v_empty[st]), ((c >> 1) - 1) & 1)) { ok = false; break; }
+        if (c >= kStages && !mbar_wait(smem_u32(&v_empty[st]), ph)) { ok = false; break; }
         const uint32_t vb_ = smem_u32(&v_full[st]);
         mbar_arrive_expect_tx(vb_, C::kVBytes);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(smem_u32(sv + kb * kBN * 128), &vmap, kb * 64, key0, kvrow, vb_);
       }
       // drain: every issued copy has been consumed before the CTA can exit
-      for (int c = max(0, nch - 2); c < nch && ok; ++c) {
-        if (!mbar_wait(smem_u32(&k_empty[c & 1]), (c >> 1) & 1) ||
-            !mbar_wait(smem_u32(&v_empty[c & 1]), (c >> 1) & 1))
+      for (int c = max(0, nch - kStages); c < nch && ok; ++c) {
+        if (!mbar_wait(smem_u32(&k_empty[c % kStages]), (c / kStages) & 1) ||
+            !mbar_wait(smem_u32(&v_empty[c % kStages]), (c / kStages) & 1))
           ok = false;
       }
       if (!ok) set_status(MD_DEV_TIMEOUT);
@@ -184,14 +206,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = umma_idesc_bf16(kBM, DH, 0, 1);
       bool ok = mbar_wait(smem_u32(q_full), 0);
       const uint32_t aq = smem_u32(sQ);
-      // S_c = Q K_c^T into TMEM buffer c & 1; frees K slot c & 1 when done
+      // S_c = Q K_c^T into TMEM buffer c % 3; frees K slot c % kStages when done.
+      // Buffer c % 3 last held P_{c-3}: P_{c-3} V_{c-3} was issued before this,
+      // and tcgen05.mma runs in issue order.
       auto issue_s = [&](int c) -> bool {
-        const int st = c & 1;
-        if (!mbar_wait(smem_u32(&k_full[st]), (c >> 1) & 1)) return false;
-        if (c >= 2 && !mbar_wait(smem_u32(&s_empty[st]), ((c >> 1) - 1) & 1)) return false;
+        const int st = c % kStages;
+        if (!mbar_wait(smem_u32(&k_full[st]), (c / kStages) & 1)) return false;
         tc_fence_after();
         const uint32_t sk = smem_u32(sKV + st * C::kStage);
-        const uint32_t d = tS + uint32_t(st * kBN);
+        const uint32_t d = tS + uint32_t((c % kSBufs) * kBN);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) {
           const uint64_t ad = umma_desc_sw128(aq + kb * kBM * 128, 16, 1024);
@@ -200,35 +223,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 4; ++kk)
             umma_f16(d, ad + uint64_t((kk * 32) >> 4), bd + uint64_t((kk * 32) >> 4), idesc_s, (kb | kk) != 0);
         }
-        umma_commit(smem_u32(&s_full[st]));
+        umma_commit(smem_u32(&s_full[c % kSBufs]));
         umma_commit(smem_u32(&k_empty[st]));
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && nch > 1) ok = issue_s(1);
+      for (int c = 0; c < kSBufs && c < nch && ok; ++c) ok = issue_s(c);
       for (int c = 0; c < nch && ok; ++c) {
-        // O += P_c V_c (hi and lo parts); frees V slot c & 1 and P when done
-        if (!mbar_wait(smem_u32(p_full), c & 1) || !mbar_wait(smem_u32(&v_full[c & 1]), (c >> 1) & 1)) {
+        // O += P_c V_c (hi and lo parts, P from TMEM); frees V slot c % kStages when done
+        const int st = c % kStages;
+        if (!mbar_wait(smem_u32(&p_full[c % kSBufs]), (c / kSBufs) & 1) ||
+            !mbar_wait(smem_u32(&v_full[st]), (c / kStages) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sv = smem_u32(sKV + (c & 1) * C::kStage + C::kKBytes);
+        const uint32_t sv = smem_u32(sKV + st * C::kStage + C::kKBytes);
+        const uint32_t tp_ = tS + uint32_t((c % kSBufs) * kBN);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t sp = smem_u32(part == 0 ? sP : sPl);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t ad =
-                umma_desc_sw128(sp + (kk >> 2) * kBM * 128, 16, 1024) + uint64_t(((kk & 3) * 32) >> 4);
             const uint64_t bd = umma_desc_sw128(sv, kBN * 128, 1024) + uint64_t((kk * 2048) >> 4);
-            umma_f16(tO, ad, bd, idesc_o, (c | part | kk) != 0);
+            umma_f16_tmem_a(tO, tp_ + uint32_t(part * (kBN / 2) + kk * 8), bd, idesc_o, (c | part | kk) != 0);
           }
         }
-        umma_commit(smem_u32(o_full));
-        umma_commit(smem_u32(&v_empty[c & 1]));
-        if (c + 2 < nch) ok = issue_s(c + 2);
+        umma_commit(smem_u32(&o_full[c & 1]));
+        umma_commit(smem_u32(&v_empty[st]));
+        if (c + kSBufs < nch) ok = issue_s(c + kSBufs);
       }
+      if (ok) umma_commit(smem_u32(o_last));
       if (!ok) set_status(MD_DEV_TIMEOUT);
     }
   } else {
@@ -241,6 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool live = grow < a.R;
     const int t = live ? grow / a.G : 0;
     const uint32_t lane_off = uint32_t(q * 32) << 16;
+    const uint64_t anc_lo = (uint64_t(tp.anc[t][1]) << 32) | tp.anc[t][0];
+    const uint64_t anc_hi = (uint64_t(tp.anc[t][3]) << 32) | tp.anc[t][2];
     const float sc = a.scale_log2;
     constexpr int kHalf = kBN / 2;
     float run_m = -INFINITY, run_l = 0.f;
@@ -248,45 +273,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every iteration runs both named barriers, so a wait that gives up (ok =
     // false) only skips work and never leaves a partner warp at a barrier.
     for (int c = 0; c < nch; ++c) {
-      if (ok && !mbar_wait(smem_u32(&s_full[c & 1]), (c >> 1) & 1)) ok = false;
+      if (ok && !mbar_wait(smem_u32(&s_full[c % kSBufs]), (c / kSBufs) & 1)) ok = false;
       ok = __all_sync(0xffffffffu, ok);          // tcgen05.ld below is warp-collective
       tc_fence_after();
-      const uint32_t sb = tS + lane_off + uint32_t((c & 1) * kBN + half * kHalf);
+      const uint32_t sbuf = tS + lane_off + uint32_t((c % kSBufs) * kBN);
       const int key0 = (c_begin + c) * kBN + half * kHalf;
       const bool plain = key0 + kHalf <= P;      // every key of this half is in the prefix
       // this half of the row's scores: one 64-column TMEM load, kept for both passes
       float s[kHalf];
       float mx = -INFINITY;
       if (ok) {
-        tmem_ld64(sb, s);
-        if (plain) {
+        tmem_ld64(sbuf + uint32_t(half * kHalf), s);
+        if (!plain) {
+          const uint64_t vis = visible_bits(anc_lo, anc_hi, key0 - P);
 #pragma unroll
-          for (int j = 0; j < kHalf; ++j) mx = fmaxf(mx, s[j]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < kHalf; ++j) {
-            const int slot = key0 + j;
-            const bool vis = slot < P || (slot < nkeys && live && tree_visible(tp, t, slot - P));
-            s[j] = vis ? s[j] : -INFINITY;
-            mx = fmaxf(mx, s[j]);
-          }
+          for (int j = 0; j < kHalf; ++j) s[j] = ((vis >> j) & 1ull) ? s[j] : -INFINITY;
         }
+        // maximum as a tree of independent pairs (short dependency chains)
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int j = 8; j < kHalf; j += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[j + i]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
-      // exchange the half maxima with the partner warp (same lane quarter)
+      // exchange the half maxima with the partner warp (same lane quarter); after
+      // the first barrier both warps have read their S columns, so either may
+      // overwrite the buffer with P
       xmax[half * kBM + r] = mx;
       named_bar_sync(1 + q, 64);
       mx = fmaxf(mx, xmax[(half ^ 1) * kBM + r]);
       named_bar_sync(1 + q, 64);                 // both have read before the slots are reused
       mx = (mx == -INFINITY) ? -INFINITY : mx * sc;
-      // The previous P V must be done before P is overwritten or O rescaled.
-      if (ok && c >= 1 && !mbar_wait(smem_u32(o_full), (c - 1) & 1)) ok = false;
-      if (!__all_sync(0xffffffffu, ok)) ok = false;   // warp-uniform from here on
       if (!ok) continue;
-      tc_fence_after();
       const bool grow_m = mx > run_m + kRescaleLog2 || (run_m == -INFINITY && mx != -INFINITY);
       const float m_new = grow_m ? mx : run_m;
       const float fold = (grow_m && run_m != -INFINITY) ? exp2f(run_m - m_new) : 1.f;
       if (__any_sync(0xffffffffu, fold != 1.f)) {   // warp-wide: tcgen05.ld/st are collective
+        // O is read and written in place: P_{c-1} V_{c-1} must have landed.
+        // S_c landing implies P_{c-3} V_{c-3} did, so o_full[(c-1) & 1] is at
+        // most one phase behind the one waited for.
+        if (c >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&o_full[(c - 1) & 1]), ((c - 1) >> 1) & 1))) {
+          ok = false;
+          continue;
+        }
+        tc_fence_after();
 #pragma unroll
         for (int e0 = half * (DH / 2); e0 < (half + 1) * (DH / 2); e0 += 32) {
           float o[32];
@@ -298,47 +331,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       run_l *= fold;
       run_m = m_new;
-      // P = exp2(S*scale - m) as bf16 hi + lo into swizzled smem (K-major over keys);
-      // masked keys hold -inf and give exactly 0
+      // P = exp2(S*scale - m) as bf16 hi + lo pairs into the S buffer; masked
+      // keys hold -inf and give exactly 0. hi is p truncated to bf16 and lo is
+      // the exact remainder p - hi truncated to bf16 (|p - hi - lo| < 2^-14 p),
+      // both taken with byte permutes instead of conversions.
       const float mb = (run_m == -INFINITY) ? 0.f : run_m;
-      float sum = 0.f;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c32 = 0; c32 < kHalf; c32 += 32) {
+      for (int g = 0; g < kHalf / 32; ++g) {     // 32 keys -> 16 columns of hi and of lo
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float p0 = exp2f(fmaf(s[c32 + j], sc, -mb));
-          const float p1 = exp2f(fmaf(s[c32 + j + 1], sc, -mb));
-          sum += p0 + p1;
-          const uint32_t h2 = pack_bf16x2(p0, p1);
-          ph[j >> 1] = h2;
-          pl[j >> 1] = pack_bf16x2(p0 - bf16lo(h2), p1 - bf16hi(h2));
+          const float p0 = exp2_sfu(fmaf(s[32 * g + j], sc, -mb));
+          const float p1 = exp2_sfu(fmaf(s[32 * g + j + 1], sc, -mb));
+          sum4[(j >> 1) & 3] += p0 + p1;
+          const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+          ph[j >> 1] = __byte_perm(u0, u1, 0x7632);
+          const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u);
+          const float r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
+          pl[j >> 1] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
         }
-        // row r, keys (half*64 + c32) .. +31 -> block `half`, 16-byte chunks c32/8 .. +3, swizzled by r%8
-        const uint32_t roff = half * kBM * 128 + r * 128;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int ch = (c32 >> 3) + g;
-          const uint32_t off = roff + ((ch ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(sP + off) = make_uint4(ph[4 * g], ph[4 * g + 1], ph[4 * g + 2], ph[4 * g + 3]);
-          *reinterpret_cast<uint4*>(sPl + off) = make_uint4(pl[4 * g], pl[4 * g + 1], pl[4 * g + 2], pl[4 * g + 3]);
-        }
+        tmem_st16u(sbuf + uint32_t(half * (kHalf / 2) + 16 * g), ph);
+        tmem_st16u(sbuf + uint32_t(kBN / 2 + half * (kHalf / 2) + 16 * g), pl);
       }
-      run_l += sum;
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      run_l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&s_empty[c & 1]));
-        mbar_arrive(smem_u32(p_full));
-      }
+      if (lane == 0) mbar_arrive(smem_u32(&p_full[c % kSBufs]));
     }
-    // this split's partial for the row: (m, l, O); each half writes its half of O
+    // This split's partial for the tile: (m, l) per row and the unnormalised O,
+    // staged through shared memory (the K/V ring is idle once the last P V has
+    // landed) so that the global writes are whole rows.
+    constexpr int kLd = DH + 4;                  // padded row: conflict-free 16-byte accesses
+    float* sO = reinterpret_cast<float*>(sKV);   // [128][kLd]
+    float* sW = sO + kBM * kLd;                  // [128][kMaxSplits + 1] merge weights, 1/L
     const size_t tile = (size_t(b) * a.Hkv + hk) * a.rtiles + rt;
     const size_t prow = (tile * a.splits + split) * kBM + r;
-    float* po = a.part_o + prow * DH;
-    if (ok && nch > 0) {
-      if (__all_sync(0xffffffffu, mbar_wait(smem_u32(o_full), (nch - 1) & 1))) {
+    const bool have_o = ok && nch > 0;
+    if (have_o) {
+      if (__all_sync(0xffffffffu, mbar_wait(smem_u32(o_last), 0))) {
         tc_fence_after();
 #pragma unroll
         for (int e0 = half * (DH / 2); e0 < (half + 1) * (DH / 2); e0 += 32) {
@@ -346,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tO + lane_off + e0, o);
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(po + e0 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            *reinterpret_cast<float4*>(sO + r * kLd + e0 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         }
       } else {
         ok = false;
@@ -357,49 +389,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(1 + q, 64);
     if (half == 0)
       a.part_ml[prow] = make_float2((ok && nch > 0) ? run_m : -INFINITY, run_l + xmax[kBM + r]);
+    named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
+    const int tid = threadIdx.x - 64;     // 0..255 over the softmax warps
+    constexpr int kF4 = DH / 4;           // float4 per row
+    if (ok && nch > 0) {
+      float* po = a.part_o + (tile * a.splits + split) * kBM * DH;
+      for (int i = tid; i < kBM * kF4; i += kSoftWarps * 32) {
+        const int row = i / kF4, c4 = i % kF4;
+        *reinterpret_cast<float4*>(po + row * DH + c4 * 4) = *reinterpret_cast<const float4*>(sO + row * kLd + c4 * 4);
+      }
+    }
 
-    // The last CTA of this (request, KV head, row tile) merges the splits in order.
+    // The last CTA of this (request, KV head, row tile) merges the splits in
+    // split order: per-row weights first, then whole rows of every split's O.
     __threadfence();
-    named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
+    named_bar_sync(5, kSoftWarps * 32);
     if (sw == 0 && lane == 0) *last_flag = (atomicAdd(&a.counters[tile], 1) == a.splits - 1);
-    named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
-    if (*last_flag && live && half == 0) {
+    named_bar_sync(5, kSoftWarps * 32);
+    if (*last_flag) {
       __threadfence();
-      const int g = grow - t * a.G;
-      float* orow = a.out + ((size_t(b) * T + t) * a.Hq + hk * a.G + g) * DH;
-      if (bad) {
-        for (int e = 0; e < DH; e += 4) *reinterpret_cast<float4*>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        const size_t base = tile * a.splits;
-        float w[kMaxSplits];
-        float mx = -INFINITY;
+      const size_t base = tile * a.splits;
+      if (half == 0) {
+        float2 ml[kMaxSplits];
 #pragma unroll
         for (int s = 0; s < kMaxSplits; ++s)
-          if (s < a.splits) mx = fmaxf(mx, __ldcg(&a.part_ml[(base + s) * kBM + r]).x);
+          ml[s] = s < a.splits ? __ldcg(&a.part_ml[(base + s) * kBM + r]) : make_float2(-INFINITY, 0.f);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kMaxSplits; ++s) mx = fmaxf(mx, ml[s].x);
         float L = 0.f;
 #pragma unroll
         for (int s = 0; s < kMaxSplits; ++s) {
-          w[s] = 0.f;
-          if (s < a.splits) {
-            const float2 ml = __ldcg(&a.part_ml[(base + s) * kBM + r]);
-            w[s] = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mx);
-            L = fmaf(ml.y, w[s], L);
-          }
+          const float w = (ml[s].x == -INFINITY) ? 0.f : exp2f(ml[s].x - mx);
+          sW[r * (kMaxSplits + 1) + s] = w;
+          L = fmaf(ml[s].y, w, L);
         }
-        const float inv = 1.f / L;
-        for (int e = 0; e < DH; e += 4) {
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        sW[r * (kMaxSplits + 1) + kMaxSplits] = 1.f / L;
+      }
+      named_bar_sync(5, kSoftWarps * 32);
+      constexpr int kU = 8;               // float4 outputs per thread and pass
+      for (int i0 = tid; i0 < kBM * kF4; i0 += kU * kSoftWarps * 32) {
+        float4 acc[kU];
 #pragma unroll
-          for (int s = 0; s < kMaxSplits; ++s) {
-            if (s < a.splits && w[s] != 0.f) {
-              const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((base + s) * kBM + r) * DH + e));
-              acc.x = fmaf(v.x, w[s], acc.x);
-              acc.y = fmaf(v.y, w[s], acc.y);
-              acc.z = fmaf(v.z, w[s], acc.z);
-              acc.w = fmaf(v.w, w[s], acc.w);
+        for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int s = 0; s < kMaxSplits; ++s) {
+          if (s < a.splits) {
+            float4 v[kU];
+            float w[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const int i = i0 + u * kSoftWarps * 32;
+              const int row = i / kF4, c4 = i % kF4;
+              w[u] = (i < kBM * kF4) ? sW[row * (kMaxSplits + 1) + s] : 0.f;
+              v[u] = w[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(
+                                       a.part_o + ((base + s) * kBM + row) * DH + c4 * 4))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              acc[u].x = fmaf(v[u].x, w[u], acc[u].x);
+              acc[u].y = fmaf(v[u].y, w[u], acc[u].y);
+              acc[u].z = fmaf(v[u].z, w[u], acc[u].z);
+              acc[u].w = fmaf(v[u].w, w[u], acc[u].w);
             }
           }
-          *reinterpret_cast<float4*>(orow + e) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i = i0 + u * kSoftWarps * 32;
+          if (i >= kBM * kF4) continue;
+          const int row = i / kF4, c4 = i % kF4;
+          const int gr = rt * kBM + row;
+          if (gr >= a.R) continue;
+          const int tt = gr / a.G, g = gr - tt * a.G;
+          float* orow = a.out + ((size_t(b) * T + tt) * a.Hq + hk * a.G + g) * DH;
+          const float inv = sW[row * (kMaxSplits + 1) + kMaxSplits];
+          *reinterpret_cast<float4*>(orow + c4 * 4) =
+              bad ? make_float4(0.f, 0.f, 0.f, 0.f)
+                  : make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
         }
       }
     }

@@ -454,10 +454,12 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 // up to kmax entries. In "partitioned" mode slot c is CTA c of the kernel that
 // produced them (the CTAs that worked on row m): that kernel split `units`
 // work units, ordered (head, column tile of `ntiles`), into contiguous CTA
-// ranges, and only CTAs whose range touches head k wrote a list. Each
-// thread gathers its slots into a sorted register list; each warp then merges
-// its 32 lists by k rounds of a shuffle arg-max over the list heads (the
-// winning lane shifts its list), and warp 0 merges the 8 warp lists the same way.
+// ranges, and only CTAs whose range touches head k wrote a list. The lists
+// that were written are compacted into shared memory (kk entries each, empty
+// entries as (-inf, INT_MAX)), padded to a power of two and bitonic-sorted in
+// the top-k order (value descending, then id ascending); the first kk entries
+// are the head's top-k. A few hundred candidates: ~40 shallow stages instead
+// of kk dependent rounds of warp arg-max.
 // ---------------------------------------------------------------------------
 struct MergeArgs {
   const float* cand_val;
@@ -470,131 +472,93 @@ struct MergeArgs {
   int kph[MD_MAX_K];
 };
 
-constexpr int kListMax = MD_MAX_KMAX;
+constexpr int kMergeCap = 4096;          // candidates per (row, head): nslots * kmax <= kMergeCap
+constexpr int kMergeThreads = 256;
 
-struct SortedList {
-  float v[kListMax];
-  int i[kListMax];
-  __device__ __forceinline__ void clear() {
-#pragma unroll
-    for (int j = 0; j < kListMax; ++j) {
-      v[j] = -INFINITY;
-      i[j] = INT_MAX;
-    }
-  }
-  __device__ __forceinline__ void push(float x, int id) {
-    if (!better(x, id, v[kListMax - 1], i[kListMax - 1])) return;
-    v[kListMax - 1] = x;
-    i[kListMax - 1] = id;
-#pragma unroll
-    for (int j = kListMax - 1; j > 0; --j) {
-      if (better(v[j], i[j], v[j - 1], i[j - 1])) {
-        const float tv = v[j]; v[j] = v[j - 1]; v[j - 1] = tv;
-        const int ti = i[j]; i[j] = i[j - 1]; i[j - 1] = ti;
-      }
-    }
-  }
-  __device__ __forceinline__ void pop() {
-#pragma unroll
-    for (int j = 0; j < kListMax - 1; ++j) {
-      v[j] = v[j + 1];
-      i[j] = i[j + 1];
-    }
-    v[kListMax - 1] = -INFINITY;
-    i[kListMax - 1] = INT_MAX;
-  }
-};
-
-// kk rounds over the warp's lists; round r's winner is returned to lane r.
-__device__ __forceinline__ void warp_merge(SortedList& L, int kk, int lane, float& out_v, int& out_i) {
-  out_v = -INFINITY;
-  out_i = INT_MAX;
-  for (int r = 0; r < kk; ++r) {
-    float bv = L.v[0];
-    int bi = L.i[0];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (better(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi != INT_MAX && L.i[0] == bi && L.v[0] == bv) L.pop();
-    if (lane == r) {
-      out_v = bv;
-      out_i = bi;
-    }
-  }
-}
-
-__global__ void __launch_bounds__(256) heads_merge_kernel(MergeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a) {
   pdl_wait_primary();          // candidates come from the previous kernel
   pdl_launch_dependents();
-  __shared__ float wv[8][kListMax];
-  __shared__ int wi[8][kListMax];
+  __shared__ float sv[kMergeCap];
+  __shared__ int si[kMergeCap];
+  __shared__ int slot_of[kMergeCap / 2];
+  __shared__ int warp_cnt[kMergeThreads / 32];
+  __shared__ int n_lists;
   const int mk = blockIdx.x;
   const int k = mk % a.K;
   const int kk = param_at(a.kph, mk % a.kh);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t base = size_t(mk) * a.nslots * a.kmax;
-  SortedList L;
-  L.clear();
-  bool first = true;
-  for (int c = threadIdx.x; c < a.nslots; c += 256) {
-    if (a.partitioned) {
+  if (threadIdx.x == 0) n_lists = 0;
+  __syncthreads();
+
+  // 1. the slots that hold a list for head k, in slot order
+  for (int c0 = 0; c0 < a.nslots; c0 += kMergeThreads) {
+    const int c = c0 + threadIdx.x;
+    bool rel = c < a.nslots;
+    if (rel && a.partitioned) {
       const long long u0 = (long long)c * a.units / a.nslots, u1 = (long long)(c + 1) * a.units / a.nslots;
-      if (u1 <= (long long)k * a.ntiles || u0 >= (long long)(k + 1) * a.ntiles) continue;
+      rel = u1 > (long long)k * a.ntiles && u0 < (long long)(k + 1) * a.ntiles;
     }
-    // a slot's list is sorted already: load it whole (independent loads)
-    float lv[kListMax];
-    int li[kListMax];
-#pragma unroll
-    for (int j = 0; j < kListMax; ++j) {
-      const bool use = j < kk;
-      lv[j] = use ? a.cand_val[base + size_t(c) * a.kmax + j] : -INFINITY;
-      li[j] = use ? a.cand_id[base + size_t(c) * a.kmax + j] : -1;
-      if (li[j] < 0) {
-        lv[j] = -INFINITY;
-        li[j] = INT_MAX;
-      }
+    const unsigned bal = __ballot_sync(0xffffffffu, rel);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int off = n_lists;
+    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
+    if (rel) slot_of[off + __popc(bal & ((1u << lane) - 1))] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = n_lists;
+      for (int w = 0; w < kMergeThreads / 32; ++w) t += warp_cnt[w];
+      n_lists = t;
     }
-    if (first) {          // the thread's first list becomes its list as it is
-#pragma unroll
-      for (int j = 0; j < kListMax; ++j) {
-        L.v[j] = lv[j];
-        L.i[j] = li[j];
-      }
-      first = false;
-    } else {
-#pragma unroll
-      for (int j = 0; j < kListMax; ++j)
-        if (li[j] != INT_MAX) L.push(lv[j], li[j]);
-    }
+    __syncthreads();
   }
-  float ov;
-  int oi;
-  warp_merge(L, kk, lane, ov, oi);
-  if (lane < kk) {
-    wv[warp][lane] = ov;
-    wi[warp][lane] = oi;
+  const int n = n_lists * kk;
+  int N = 32;
+  while (N < n) N <<= 1;
+
+  // 2. gather (value, id) pairs; pad with (-inf, INT_MAX)
+  for (int e = threadIdx.x; e < N; e += kMergeThreads) {
+    float v = -INFINITY;
+    int id = INT_MAX;
+    if (e < n) {
+      const int c = slot_of[e / kk], j = e % kk;
+      const size_t at = base + size_t(c) * a.kmax + j;
+      const int x = a.cand_id[at];
+      if (x >= 0) {
+        v = a.cand_val[at];
+        id = x;
+      }
+    }
+    sv[e] = v;
+    si[e] = id;
   }
   __syncthreads();
-  if (warp == 0) {
-    // lane l takes warp l's merged list (sorted) as it is
-#pragma unroll
-    for (int j = 0; j < kListMax; ++j) {
-      const bool use = lane < 8 && j < kk;
-      L.v[j] = use ? wv[lane][j] : -INFINITY;
-      L.i[j] = use ? wi[lane][j] : INT_MAX;
+
+  // 3. bitonic sort, best first
+  for (int size = 2; size <= N; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < (N >> 1); t += kMergeThreads) {
+        const int i = 2 * t - (t & (stride - 1));     // lower index of the pair
+        const int j = i + stride;
+        const bool desc = (i & size) == 0;            // this run is ordered best first
+        const float vi = sv[i], vj = sv[j];
+        const int ii = si[i], ij = si[j];
+        if (better(vj, ij, vi, ii) == desc) {
+          sv[i] = vj; si[i] = ij;
+          sv[j] = vi; si[j] = ii;
+        }
+      }
+      __syncthreads();
     }
-    warp_merge(L, kk, lane, ov, oi);
-    if (lane < a.kmax) {
-      const bool used = lane < kk && oi != INT_MAX;
-      a.topk_vals[size_t(mk) * a.kmax + lane] = used ? ov : -INFINITY;
-      a.topk_ids[size_t(mk) * a.kmax + lane] = used ? oi : -1;
-    }
+  }
+
+  // 4. the first kk entries; the rest of the kmax slots are empty
+  if (threadIdx.x < a.kmax) {
+    const int r = threadIdx.x;
+    const bool used = r < kk && r < N && si[r] != INT_MAX;
+    a.topk_vals[size_t(mk) * a.kmax + r] = used ? sv[r] : -INFINITY;
+    a.topk_ids[size_t(mk) * a.kmax + r] = used ? si[r] : -1;
   }
 }
 
