@@ -118,11 +118,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
   float* xmax = reinterpret_cast<float*>(bars + 32);    // [2 halves][128 rows] chunk maxima
 
-  const int split = blockIdx.x, rt = blockIdx.y % a.rtiles, hk = blockIdx.y / a.rtiles, b = blockIdx.z;
+  const int split = blockIdx.x, rt = blockIdx.y % a.rtiles, hk = blockIdx.y / a.rtiles;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = tp.T;
   pdl_wait_primary();          // inputs may come from earlier kernels
   pdl_launch_dependents();
+  // Blocks are launched in index order, so blockIdx.z walks the requests from
+  // the longest prefix down (ties by index): long tiles start first and short
+  // ones fill the tail. Warp 0 finds the request of rank blockIdx.z.
+  int* req = last_flag + 1;
+  if (warp == 0) {
+    for (int c = lane; c < a.B; c += 32) {
+      const int pc = a.prefix_len[c];
+      int rank = 0;
+      for (int j = 0; j < a.B; ++j) {
+        const int pj = a.prefix_len[j];
+        rank += (pj > pc || (pj == pc && j < c)) ? 1 : 0;
+      }
+      if (rank == int(blockIdx.z)) *req = c;
+    }
+  }
+  __syncthreads();
+  const int b = *req;
   const int P = a.prefix_len[b];
   const bool bad = P < 0 || P + T > a.S_max;
   const int nkeys = bad ? 0 : P + T;
@@ -387,87 +404,107 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) set_status(MD_DEV_TIMEOUT);
     xmax[half * kBM + r] = run_l;
     named_bar_sync(1 + q, 64);
-    if (half == 0)
-      a.part_ml[prow] = make_float2((ok && nch > 0) ? run_m : -INFINITY, run_l + xmax[kBM + r]);
-    named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
+    const float l_row = run_l + xmax[(half ^ 1) * kBM + r];
     const int tid = threadIdx.x - 64;     // 0..255 over the softmax warps
     constexpr int kF4 = DH / 4;           // float4 per row
-    if (ok && nch > 0) {
-      float* po = a.part_o + (tile * a.splits + split) * kBM * DH;
+    if (a.splits == 1) {
+      // one split: the tile's rows are final, written straight from shared memory
+      if (half == 0) sW[r * (kMaxSplits + 1) + kMaxSplits] = 1.f / l_row;
+      named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
       for (int i = tid; i < kBM * kF4; i += kSoftWarps * 32) {
         const int row = i / kF4, c4 = i % kF4;
-        *reinterpret_cast<float4*>(po + row * DH + c4 * 4) = *reinterpret_cast<const float4*>(sO + row * kLd + c4 * 4);
-      }
-    }
-
-    // The last CTA of this (request, KV head, row tile) merges the splits in
-    // split order: per-row weights first, then whole rows of every split's O.
-    __threadfence();
-    named_bar_sync(5, kSoftWarps * 32);
-    if (sw == 0 && lane == 0) *last_flag = (atomicAdd(&a.counters[tile], 1) == a.splits - 1);
-    named_bar_sync(5, kSoftWarps * 32);
-    if (*last_flag) {
-      __threadfence();
-      const size_t base = tile * a.splits;
-      if (half == 0) {
-        float2 ml[kMaxSplits];
-#pragma unroll
-        for (int s = 0; s < kMaxSplits; ++s)
-          ml[s] = s < a.splits ? __ldcg(&a.part_ml[(base + s) * kBM + r]) : make_float2(-INFINITY, 0.f);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < kMaxSplits; ++s) mx = fmaxf(mx, ml[s].x);
-        float L = 0.f;
-#pragma unroll
-        for (int s = 0; s < kMaxSplits; ++s) {
-          const float w = (ml[s].x == -INFINITY) ? 0.f : exp2f(ml[s].x - mx);
-          sW[r * (kMaxSplits + 1) + s] = w;
-          L = fmaf(ml[s].y, w, L);
+        const int gr = rt * kBM + row;
+        if (gr >= a.R) continue;
+        const int tt = gr / a.G, g = gr - tt * a.G;
+        float* orow = a.out + ((size_t(b) * T + tt) * a.Hq + hk * a.G + g) * DH;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ok && nch > 0 && !bad) {
+          const float inv = sW[row * (kMaxSplits + 1) + kMaxSplits];
+          v = *reinterpret_cast<const float4*>(sO + row * kLd + c4 * 4);
+          v = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
         }
-        sW[r * (kMaxSplits + 1) + kMaxSplits] = 1.f / L;
+        *reinterpret_cast<float4*>(orow + c4 * 4) = v;
       }
+    } else {
+      if (half == 0) a.part_ml[prow] = make_float2((ok && nch > 0) ? run_m : -INFINITY, l_row);
+      named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
+      if (ok && nch > 0) {
+        float* po = a.part_o + (tile * a.splits + split) * kBM * DH;
+        for (int i = tid; i < kBM * kF4; i += kSoftWarps * 32) {
+          const int row = i / kF4, c4 = i % kF4;
+          *reinterpret_cast<float4*>(po + row * DH + c4 * 4) = *reinterpret_cast<const float4*>(sO + row * kLd + c4 * 4);
+        }
+      }
+
+      // The last CTA of this (request, KV head, row tile) merges the splits in
+      // split order: per-row weights first, then whole rows of every split's O.
+      __threadfence();
       named_bar_sync(5, kSoftWarps * 32);
-      constexpr int kU = 8;               // float4 outputs per thread and pass
-      for (int i0 = tid; i0 < kBM * kF4; i0 += kU * kSoftWarps * 32) {
-        float4 acc[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int s = 0; s < kMaxSplits; ++s) {
-          if (s < a.splits) {
-            float4 v[kU];
-            float w[kU];
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-              const int i = i0 + u * kSoftWarps * 32;
-              const int row = i / kF4, c4 = i % kF4;
-              w[u] = (i < kBM * kF4) ? sW[row * (kMaxSplits + 1) + s] : 0.f;
-              v[u] = w[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(
-                                       a.part_o + ((base + s) * kBM + row) * DH + c4 * 4))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-              acc[u].x = fmaf(v[u].x, w[u], acc[u].x);
-              acc[u].y = fmaf(v[u].y, w[u], acc[u].y);
-              acc[u].z = fmaf(v[u].z, w[u], acc[u].z);
-              acc[u].w = fmaf(v[u].w, w[u], acc[u].w);
+      if (sw == 0 && lane == 0) *last_flag = (atomicAdd(&a.counters[tile], 1) == a.splits - 1);
+      named_bar_sync(5, kSoftWarps * 32);
+      if (*last_flag) {
+        __threadfence();
+        const size_t base = tile * a.splits;
+        if (half == 0) {
+          float2 ml[kMaxSplits];
+  #pragma unroll
+          for (int s = 0; s < kMaxSplits; ++s)
+            ml[s] = s < a.splits ? __ldcg(&a.part_ml[(base + s) * kBM + r]) : make_float2(-INFINITY, 0.f);
+          float mx = -INFINITY;
+  #pragma unroll
+          for (int s = 0; s < kMaxSplits; ++s) mx = fmaxf(mx, ml[s].x);
+          float L = 0.f;
+  #pragma unroll
+          for (int s = 0; s < kMaxSplits; ++s) {
+            const float w = (ml[s].x == -INFINITY) ? 0.f : exp2f(ml[s].x - mx);
+            sW[r * (kMaxSplits + 1) + s] = w;
+            L = fmaf(ml[s].y, w, L);
+          }
+          sW[r * (kMaxSplits + 1) + kMaxSplits] = 1.f / L;
+        }
+        named_bar_sync(5, kSoftWarps * 32);
+        constexpr int kU = 8;               // float4 outputs per thread and pass
+        for (int i0 = tid; i0 < kBM * kF4; i0 += kU * kSoftWarps * 32) {
+          float4 acc[kU];
+  #pragma unroll
+          for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  #pragma unroll
+          for (int s = 0; s < kMaxSplits; ++s) {
+            if (s < a.splits) {
+              float4 v[kU];
+              float w[kU];
+  #pragma unroll
+              for (int u = 0; u < kU; ++u) {
+                const int i = i0 + u * kSoftWarps * 32;
+                const int row = i / kF4, c4 = i % kF4;
+                w[u] = (i < kBM * kF4) ? sW[row * (kMaxSplits + 1) + s] : 0.f;
+                v[u] = w[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(
+                                         a.part_o + ((base + s) * kBM + row) * DH + c4 * 4))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+  #pragma unroll
+              for (int u = 0; u < kU; ++u) {
+                acc[u].x = fmaf(v[u].x, w[u], acc[u].x);
+                acc[u].y = fmaf(v[u].y, w[u], acc[u].y);
+                acc[u].z = fmaf(v[u].z, w[u], acc[u].z);
+                acc[u].w = fmaf(v[u].w, w[u], acc[u].w);
+              }
             }
           }
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int i = i0 + u * kSoftWarps * 32;
-          if (i >= kBM * kF4) continue;
-          const int row = i / kF4, c4 = i % kF4;
-          const int gr = rt * kBM + row;
-          if (gr >= a.R) continue;
-          const int tt = gr / a.G, g = gr - tt * a.G;
-          float* orow = a.out + ((size_t(b) * T + tt) * a.Hq + hk * a.G + g) * DH;
-          const float inv = sW[row * (kMaxSplits + 1) + kMaxSplits];
-          *reinterpret_cast<float4*>(orow + c4 * 4) =
-              bad ? make_float4(0.f, 0.f, 0.f, 0.f)
-                  : make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
+  #pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kSoftWarps * 32;
+            if (i >= kBM * kF4) continue;
+            const int row = i / kF4, c4 = i % kF4;
+            const int gr = rt * kBM + row;
+            if (gr >= a.R) continue;
+            const int tt = gr / a.G, g = gr - tt * a.G;
+            float* orow = a.out + ((size_t(b) * T + tt) * a.Hq + hk * a.G + g) * DH;
+            const float inv = sW[row * (kMaxSplits + 1) + kMaxSplits];
+            *reinterpret_cast<float4*>(orow + c4 * 4) =
+                bad ? make_float4(0.f, 0.f, 0.f, 0.f)
+                    : make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
+          }
         }
       }
     }

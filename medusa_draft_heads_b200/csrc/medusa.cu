@@ -502,7 +502,9 @@ AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
   p.R = T * p.G;
   p.tc = (128 % p.G) == 0;
   if (p.tc) {
-    // one wave of CTAs: (splits x row tiles x KV heads x requests) <= #SMs
+    // One wave of CTAs: (splits x row tiles x KV heads x requests) <= #SMs.
+    // (Finer splits that even out unequal prefix lengths measured slower: every
+    // CTA pays a prologue and epilogue of a few chunks' time and the merge.)
     p.rtiles = (p.R + 127) / 128;
     const int chunks = (S_max + md::attn_tc::kBN - 1) / md::attn_tc::kBN;
     const int base = B * Hkv * p.rtiles;
