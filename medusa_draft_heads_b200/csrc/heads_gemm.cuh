@@ -21,15 +21,14 @@
 // Work split: the grid is mtiles groups of per_mt CTAs, group g takes row
 // tile g, and CTA j of every group takes the same contiguous range
 // [j*U/per_mt, (j+1)*U/per_mt) of the U = K * ntiles (head, column tile)
-// units. The CTAs with the same j therefore walk the same weight strips in
-// step: a strip comes from HBM once and from L2 for the other row tiles, and
-// the strips in flight at any moment (per_mt of them) fit in L2. (Contiguous
-// ranges over all tiles would put the CTAs of different row tiles on
-// different strips at any one time; with mtiles x per_mt strips in flight the
-// reuse distance exceeds L2 and every row tile re-reads its strips from HBM.)
-// In phase 2 each row keeps one running top-k across the CTA's column tiles:
-// after the first tiles nearly every logit is rejected by one compare against
-// the current k-th best.
+// units, so the CTAs that share a weight strip read it at about the same time
+// and the strips in flight at any moment number per_mt. (Contiguous ranges
+// over all tiles put the CTAs of different row tiles on different strips and
+// measured 5x the weight bytes from HBM at 520 rows.) The launcher uses this
+// kernel up to 128 rows (one row tile); beyond that the CTA-pair kernel of
+// heads_gemm2.cuh. In phase 2 each row keeps one running top-k across the
+// CTA's column tiles: after the first tiles nearly every logit is rejected by
+// one compare against the current k-th best.
 #pragma once
 
 #include "common.cuh"

@@ -476,7 +476,20 @@ AcceptPlan accept_plan(int B, int T, int V) {
   AcceptPlan p;
   const int rows = B * T;
   const int max_chunks = (V + 1023) / 1024;
-  int n = (4 * num_sms() + rows - 1) / rows;      // ~4 CTAs per SM: enough loads in flight
+  // as many row chunks as fit one wave of resident CTAs (~4 per SM: enough
+  // loads in flight), so that no second partial wave trails the scan
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, md::acc::accept_rows_kernel, md::acc::kRowThreads, 0) !=
+            cudaSuccess ||
+        nb <= 0) {
+      cudaGetLastError();
+      nb = 4;
+    }
+    per_sm = nb;
+  }
+  int n = per_sm * num_sms() / rows;
   n = std::max(1, std::min(n, max_chunks));
   int len = (V + n - 1) / n;
   len = (len + 1023) / 1024 * 1024;
