@@ -50,6 +50,41 @@ def heads_bytes(w):
     return w.head_weight_bytes() + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax
 
 
+TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                               "heads_traffic_prof-8b-v32000.md")
+HEADS_SOURCES = ("heads.cuh", "common.cuh")
+
+
+def heads_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in HEADS_SOURCES:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "medusa_draft_heads_b200", "csrc", f),
+                  "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_heads_traffic(w):
+    """DRAM bytes of one streaming heads call: the ratio DRAM traffic /
+    algorithmic bytes recorded from an ncu capture (profiles/
+    heads_traffic_prof-8b-v32000.md) times this workload's algorithmic bytes.
+    None on the tensor-core path, or when the heads sources changed since the
+    capture (digest mismatch)."""
+    if w.M > 4 or not os.path.exists(TRAFFIC_PROFILE):
+        return None
+    ratio = digest = None
+    with open(TRAFFIC_PROFILE) as fh:
+        for line in fh:
+            if line.startswith("traffic_per_algorithmic_byte:"):
+                ratio = float(line.split(":")[1])
+            elif line.startswith("heads_source_digest:"):
+                digest = line.split(":")[1].split()[0]
+    if ratio is None or digest != heads_source_digest():
+        return None
+    return ratio * heads_bytes(w)
+
+
 def slowest_rank_ms(ms: float, world: int, device=None) -> float:
     """Elapsed milliseconds of the slowest rank (all-reduce MAX; a no-op on one rank)."""
     if world <= 1:
@@ -409,7 +444,7 @@ def run_medusa(args, w):
         hb = heads_bytes(w)
         hf = heads_flops(w)
         heads_ms = float(per_call[:, 0].mean())
-        if w.M > 8:      # tensor-core GEMM path: bound by the bf16 tensor pipe
+        if w.M > 4:      # tensor-core GEMM path: bound by the bf16 tensor pipe
             roof = {"kernel": "md_medusa_heads (tcgen05 GEMMs: residual block, vocabulary projection + top-k; merge)",
                     "bound": "tensor", "achieved": hf / (heads_ms / 1000.0) / 1e12,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
@@ -419,7 +454,10 @@ def run_medusa(args, w):
                     "bound": "hbm", "achieved": hb / (heads_ms / 1000.0) / 1e9, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "algorithmic_bytes": hb, "peak_note": "measured copy bandwidth"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = args.traffic
+        roof["traffic"] = args.traffic if args.traffic is not None else measured_heads_traffic(w)
+        roof["traffic_source"] = ("--traffic" if args.traffic is not None else
+                                  "profiles/heads_traffic_prof-8b-v32000.md scaled by algorithmic bytes"
+                                  if roof["traffic"] is not None else None)
         roof["avg_ms"] = heads_ms
         roof["peak_source"] = peaks["source"]
         ab = attention_bytes(w, P)
