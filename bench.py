@@ -650,7 +650,8 @@ def run_sweep(args):
                     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
                     tot = float(np.mean([e[0].elapsed_time(e[4]) for e in evs]))
                     print(json.dumps({"sweep": w.name, "B": B, "tree": tree, "prefix": P, "mode": mode,
-                                      "heads_path": "tcgen05-gemm" if w.M > 8 else "cuda-core-stream",
+                                      "heads_path": ("tcgen05-pair-gemm" if w.M > 128 else "tcgen05-gemm" if w.M > 4
+                                                     else "cuda-core-stream"),
                                       "steps_per_s": 1000.0 / tot, "ms_per_step": tot,
                                       "ms": {"heads": float(per[:, 0].mean()), "build": float(per[:, 1].mean()),
                                              "attention": float(per[:, 2].mean()),
