@@ -32,9 +32,12 @@
 // are computed while the softmax works on c: the softmax warps and the tensor
 // pipe work on different chunks at the same time.
 //
-// Each CTA writes its split's (m, sum, unnormalised O) per row; the last CTA of
-// a (request, KV head, row tile) to finish combines the splits in split order
-// and writes the output rows.
+// The KV splits of one (request, KV head, row tile) are the CTAs of one
+// cluster. Each stages its split's unnormalised O and per-row (m, sum) in its
+// shared memory; after a cluster barrier every CTA combines its share of the
+// rows from all splits' shared memory (distributed shared memory loads, in
+// split order) and writes them; a second cluster barrier keeps each CTA's
+// shared memory alive until its peers are done reading it.
 #pragma once
 
 #include "common.cuh"
@@ -48,7 +51,7 @@ constexpr int kSoftWarps = 8;
 constexpr int kThreads = 64 + kSoftWarps * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;   // lazy rescale threshold (factor 256)
-constexpr int kMaxSplits = 16;
+constexpr int kMaxSplits = 8;    // KV splits of one tile = CTAs of one cluster (portable size)
 
 constexpr int kStages = 3;      // K / V ring depth
 constexpr int kSBufs = 3;       // S / P buffers in TMEM (3 x 128 columns + O)
@@ -61,13 +64,12 @@ struct Cfg {
   static constexpr uint32_t kVBytes = KB * kBN * 128;         // V chunk, N(dh)-major SW128
   static constexpr uint32_t kStage = kKBytes + kVBytes;
   static constexpr int kSmem = kQBytes + kStages * kStage + 1024 + 256 + 1024;  // + barriers, maxima
+  // the epilogue stages O, the merge weights and (m, l) over the idle K/V ring
+  static_assert(kBM * (DH + 4) * 4 + kBM * (kMaxSplits + 1) * 4 + kBM * 8 <= kStages * kStage, "staging");
 };
 
 struct Args {
   const int32_t* prefix_len;  // [B]
-  float* part_o;              // [B, Hkv, rtiles, splits, 128, dh]
-  float2* part_ml;            // [B, Hkv, rtiles, splits, 128]   (max, sum) in log2 units
-  int* counters;              // [B, Hkv, rtiles], zero before the launch
   float* out;                 // [B, T, Hq, dh]
   int B, S_max, Hq, Hkv, G, R, rtiles, splits, chunks_per_split;
   float scale_log2;
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = p_full + kSBufs;           // 2: P_c V_c commits to o_full[c & 1]
   uint64_t* o_last = o_full + 2;                // 1: every P V done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + 1);
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
+  int* req = reinterpret_cast<int*>(tmem_slot + 2);   // request served by this CTA
   float* xmax = reinterpret_cast<float*>(bars + 32);    // [2 halves][128 rows] chunk maxima
 
   const int split = blockIdx.x, rt = blockIdx.y % a.rtiles, hk = blockIdx.y / a.rtiles;
@@ -126,7 +128,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Blocks are launched in index order, so blockIdx.z walks the requests from
   // the longest prefix down (ties by index): long tiles start first and short
   // ones fill the tail. Warp 0 finds the request of rank blockIdx.z.
-  int* req = last_flag + 1;
   if (warp == 0) {
     for (int c = lane; c < a.B; c += 32) {
       const int pc = a.prefix_len[c];
@@ -179,6 +180,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tO = tmem + kSBufs * kBN;  // O at columns [384, 384 + DH)
   const int kvrow = b * a.Hkv + hk;
   const int tpt = kBM / a.G;                // tree tokens per query tile
+  // epilogue staging over the K/V ring: O [128][kLd] (padded rows: conflict-free
+  // 16-byte accesses), merge weights [128][kMaxSplits + 1] (1/L last), (m, l) [128]
+  constexpr int kLd = DH + 4;
+  float* sO = reinterpret_cast<float*>(sKV);
+  float* sW = sO + kBM * kLd;
+  float2* sML = reinterpret_cast<float2*>(sW + kBM * (kMaxSplits + 1));
 
   if (warp == 0) {
     // ---------------------------------- TMA ----------------------------------
@@ -377,14 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&p_full[c % kSBufs]));
     }
-    // This split's partial for the tile: (m, l) per row and the unnormalised O,
-    // staged through shared memory (the K/V ring is idle once the last P V has
-    // landed) so that the global writes are whole rows.
-    constexpr int kLd = DH + 4;                  // padded row: conflict-free 16-byte accesses
-    float* sO = reinterpret_cast<float*>(sKV);   // [128][kLd]
-    float* sW = sO + kBM * kLd;                  // [128][kMaxSplits + 1] merge weights, 1/L
-    const size_t tile = (size_t(b) * a.Hkv + hk) * a.rtiles + rt;
-    const size_t prow = (tile * a.splits + split) * kBM + r;
+    // This split's unnormalised O and (m, l) per row, staged in shared memory
+    // (the K/V ring is idle once the last P V has landed).
     const bool have_o = ok && nch > 0;
     if (have_o) {
       if (__all_sync(0xffffffffu, mbar_wait(smem_u32(o_last), 0))) {
@@ -425,89 +426,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<float4*>(orow + c4 * 4) = v;
       }
-    } else {
-      if (half == 0) a.part_ml[prow] = make_float2((ok && nch > 0) ? run_m : -INFINITY, l_row);
-      named_bar_sync(5, kSoftWarps * 32);   // ids 1..4: partner pairs
-      if (ok && nch > 0) {
-        float* po = a.part_o + (tile * a.splits + split) * kBM * DH;
-        for (int i = tid; i < kBM * kF4; i += kSoftWarps * 32) {
-          const int row = i / kF4, c4 = i % kF4;
-          *reinterpret_cast<float4*>(po + row * DH + c4 * 4) = *reinterpret_cast<const float4*>(sO + row * kLd + c4 * 4);
-        }
-      }
+    } else if (half == 0) {
+      sML[r] = make_float2(have_o ? run_m : -INFINITY, l_row);
+    }
+  }
 
-      // The last CTA of this (request, KV head, row tile) merges the splits in
-      // split order: per-row weights first, then whole rows of every split's O.
-      __threadfence();
-      named_bar_sync(5, kSoftWarps * 32);
-      if (sw == 0 && lane == 0) *last_flag = (atomicAdd(&a.counters[tile], 1) == a.splits - 1);
-      named_bar_sync(5, kSoftWarps * 32);
-      if (*last_flag) {
-        __threadfence();
-        const size_t base = tile * a.splits;
-        if (half == 0) {
-          float2 ml[kMaxSplits];
-  #pragma unroll
-          for (int s = 0; s < kMaxSplits; ++s)
-            ml[s] = s < a.splits ? __ldcg(&a.part_ml[(base + s) * kBM + r]) : make_float2(-INFINITY, 0.f);
-          float mx = -INFINITY;
-  #pragma unroll
-          for (int s = 0; s < kMaxSplits; ++s) mx = fmaxf(mx, ml[s].x);
-          float L = 0.f;
-  #pragma unroll
-          for (int s = 0; s < kMaxSplits; ++s) {
-            const float w = (ml[s].x == -INFINITY) ? 0.f : exp2f(ml[s].x - mx);
-            sW[r * (kMaxSplits + 1) + s] = w;
-            L = fmaf(ml[s].y, w, L);
-          }
-          sW[r * (kMaxSplits + 1) + kMaxSplits] = 1.f / L;
+  if (a.splits > 1) {
+    // ------------------- split merge through distributed shared memory -------------------
+    __syncwarp();
+    cluster_sync();                      // every split of the tile is staged
+    if (warp >= 2) {
+      const int tid = threadIdx.x - 64;
+      const uint32_t crank = cluster_ctarank();
+      const int r0 = int(crank) * kBM / a.splits, r1 = int(crank + 1) * kBM / a.splits;
+      // per-row weights of each split and 1/L for this CTA's rows
+      for (int i = tid; i < r1 - r0; i += kSoftWarps * 32) {
+        const int row = r0 + i;
+        float2 ml[kMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplits; ++sp)
+          ml[sp] = sp < a.splits ? ld_cluster_f2(mapa_shared(smem_u32(&sML[row]), uint32_t(sp)))
+                                 : make_float2(-INFINITY, 0.f);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplits; ++sp) mx = fmaxf(mx, ml[sp].x);
+        float L = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplits; ++sp) {
+          const float w = (ml[sp].x == -INFINITY) ? 0.f : exp2f(ml[sp].x - mx);
+          sW[row * (kMaxSplits + 1) + sp] = w;
+          L = fmaf(ml[sp].y, w, L);
         }
-        named_bar_sync(5, kSoftWarps * 32);
-        constexpr int kU = 8;               // float4 outputs per thread and pass
-        for (int i0 = tid; i0 < kBM * kF4; i0 += kU * kSoftWarps * 32) {
-          float4 acc[kU];
-  #pragma unroll
-          for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-  #pragma unroll
-          for (int s = 0; s < kMaxSplits; ++s) {
-            if (s < a.splits) {
-              float4 v[kU];
-              float w[kU];
-  #pragma unroll
-              for (int u = 0; u < kU; ++u) {
-                const int i = i0 + u * kSoftWarps * 32;
-                const int row = i / kF4, c4 = i % kF4;
-                w[u] = (i < kBM * kF4) ? sW[row * (kMaxSplits + 1) + s] : 0.f;
-                v[u] = w[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(
-                                         a.part_o + ((base + s) * kBM + row) * DH + c4 * 4))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-  #pragma unroll
-              for (int u = 0; u < kU; ++u) {
-                acc[u].x = fmaf(v[u].x, w[u], acc[u].x);
-                acc[u].y = fmaf(v[u].y, w[u], acc[u].y);
-                acc[u].z = fmaf(v[u].z, w[u], acc[u].z);
-                acc[u].w = fmaf(v[u].w, w[u], acc[u].w);
-              }
-            }
-          }
-  #pragma unroll
+        sW[row * (kMaxSplits + 1) + kMaxSplits] = 1.f / L;
+      }
+      named_bar_sync(5, kSoftWarps * 32);
+      constexpr int kF4 = DH / 4;
+      constexpr int kU = 2;               // float4 outputs per thread and pass: all loads of a pass in flight
+      const int n4 = (r1 - r0) * kF4;
+      for (int i0 = tid; i0 < n4; i0 += kU * kSoftWarps * 32) {
+        float4 v[kMaxSplits][kU];
+        float w[kMaxSplits][kU];
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplits; ++sp)
+#pragma unroll
           for (int u = 0; u < kU; ++u) {
             const int i = i0 + u * kSoftWarps * 32;
-            if (i >= kBM * kF4) continue;
-            const int row = i / kF4, c4 = i % kF4;
-            const int gr = rt * kBM + row;
-            if (gr >= a.R) continue;
-            const int tt = gr / a.G, g = gr - tt * a.G;
-            float* orow = a.out + ((size_t(b) * T + tt) * a.Hq + hk * a.G + g) * DH;
-            const float inv = sW[row * (kMaxSplits + 1) + kMaxSplits];
-            *reinterpret_cast<float4*>(orow + c4 * 4) =
-                bad ? make_float4(0.f, 0.f, 0.f, 0.f)
-                    : make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
+            const int row = r0 + i / kF4, c4 = i % kF4;
+            w[sp][u] = (sp < a.splits && i < n4 && !bad) ? sW[row * (kMaxSplits + 1) + sp] : 0.f;
+            v[sp][u] = w[sp][u] != 0.f ? ld_cluster_f4(mapa_shared(smem_u32(sO + row * kLd + c4 * 4), uint32_t(sp)))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i = i0 + u * kSoftWarps * 32;
+          if (i >= n4) continue;
+          const int row = r0 + i / kF4, c4 = i % kF4;
+          const int gr = rt * kBM + row;
+          if (gr >= a.R) continue;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int sp = 0; sp < kMaxSplits; ++sp) {
+            acc.x = fmaf(v[sp][u].x, w[sp][u], acc.x);
+            acc.y = fmaf(v[sp][u].y, w[sp][u], acc.y);
+            acc.z = fmaf(v[sp][u].z, w[sp][u], acc.z);
+            acc.w = fmaf(v[sp][u].w, w[sp][u], acc.w);
+          }
+          const float inv = bad ? 0.f : sW[row * (kMaxSplits + 1) + kMaxSplits];
+          const int tt = gr / a.G, g = gr - tt * a.G;
+          *reinterpret_cast<float4*>(a.out + ((size_t(b) * T + tt) * a.Hq + hk * a.G + g) * DH + c4 * 4) =
+              make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         }
       }
     }
+    __syncwarp();
+    cluster_sync();                      // peers are done reading this CTA's shared memory
   }
   tc_fence_before();
   __syncthreads();

@@ -526,10 +526,8 @@ AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
     p.cps = (chunks + splits - 1) / splits;
     p.splits = (chunks + p.cps - 1) / p.cps;
     p.max_chunks = chunks;
-    const size_t rows = size_t(base) * p.splits * 128;
-    p.off_ml = align256(rows * dh * 4);
-    p.off_cnt = p.off_ml + align256(rows * 8);
-    p.bytes = p.off_cnt + align256(size_t(base) * 4);
+    p.off_ml = p.off_cnt = 0;
+    p.bytes = 256;          // the splits merge through distributed shared memory: no scratch
   } else {
     p.rtiles = p.splits = p.cps = 0;
     p.max_chunks = (S_max + md::attn::kChunk - 1) / md::attn::kChunk;
@@ -563,21 +561,31 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   }
   if ((s = make_map_3d_sw128(&kmap, kc, DH, S_max, uint64_t(B) * Hkv, 64, kBN)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&vmap, vc, DH, S_max, uint64_t(B) * Hkv, 64, kBN)) != MD_OK) return s;
+  (void)ws;
   Args a;
   a.prefix_len = prefix_len;
-  a.part_o = static_cast<float*>(ws);
-  a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
-  a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pl.off_cnt);
   a.out = out;
   a.B = B; a.S_max = S_max; a.Hq = Hq; a.Hkv = Hkv; a.G = pl.G; a.R = pl.R; a.rtiles = pl.rtiles;
   a.splits = pl.splits; a.chunks_per_split = pl.cps;
   a.scale_log2 = sc * 1.4426950408889634f;
-  if ((s = cuda_ok(cudaMemsetAsync(a.counters, 0, size_t(B) * Hkv * pl.rtiles * 4, st))) != MD_OK) return s;
   constexpr int sm = Cfg<DH>::kSmem;
   if ((s = set_smem(attn_tc_kernel<DH>, sm)) != MD_OK) return s;
-  // ordinary launch: the counters were just zeroed by a memset on this stream
-  attn_tc_kernel<DH><<<dim3(pl.splits, Hkv * pl.rtiles, B), kThreads, sm, st>>>(qmap, kmap, vmap, tree->tp, a);
-  return last_launch();
+  // the KV splits of a tile form one cluster (they merge through its shared memory)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.splits, Hkv * pl.rtiles, B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pl.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, attn_tc_kernel<DH>, qmap, kmap, vmap, tree->tp, a));
 }
 
 // Scratch of md_medusa_heads_static: a fixed array in the library's device
