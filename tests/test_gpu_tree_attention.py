@@ -122,14 +122,21 @@ def test_tree_attention_70b_sampled_rows():
         assert normwise(out[b, t, h], ref[b, t, h]) <= ATTN_RTOL
 
 
-def test_tree_attention_bad_prefix_sets_status_and_zeros():
+@pytest.mark.parametrize("S_max", [128, 1024])
+def test_tree_attention_bad_prefix_sets_status_and_zeros(S_max):
+    """A prefix that leaves no room for the tree zeroes that request only. With
+    S_max = 1024 the key range is cut into 8 splits (one cluster per tile):
+    the bad request's splits all hold nothing, and the good request's keys
+    fall in its first split only."""
     tups = ot.select_tree((4, 3, 2, 2), TREE_ACCEPT, 16)
     md.device_status(clear=True)
-    out, _ = _attention_case(3, tups, 2, 4, 2, 64, np.array([100, 60]), 128)   # 100 + 17 <= 128: valid
+    out, _ = _attention_case(3, tups, 2, 4, 2, 64, np.array([S_max - 28, 60]), S_max)   # P + 17 <= S_max: valid
     assert md.device_status(clear=True) == 0
-    out, _ = _attention_case(3, tups, 2, 4, 2, 64, np.array([120, 60]), 128)   # 120 + 17 > 128
+    out, (q, k, v, parent) = _attention_case(3, tups, 2, 4, 2, 64, np.array([S_max - 8, 60]), S_max)  # P + 17 > S_max
     assert md.device_status(clear=True) == md.binding.DEV_BAD_PREFIX
     assert np.all(out[0] == 0) and np.all(np.isfinite(out[1])) and np.any(out[1] != 0)
+    ref = oa.tree_attention(q[1:], k[1:], v[1:], np.array([60]), parent)
+    assert normwise(out[1:], ref).max() <= ATTN_RTOL
 
 
 def test_tree_attention_explicit_scale_and_determinism():
