@@ -26,7 +26,7 @@ constexpr int kConsumerWarps = 8;   // phase-2 math warps (one more warp feeds T
 constexpr int kZPad = 8;            // z row i is stored as 8 bf16 (one per m), 16 B
 constexpr int kW1Threads = 256;
 constexpr int kW1TileO = 256;       // phase-1 output columns per CTA
-constexpr int kW1MaxRows = 1024;    // phase-1 hidden rows per CTA (split-K)
+constexpr int kW1MaxRows = 2048;    // phase-1 hidden rows per CTA (split-K)
 constexpr int kMaxM = 4;        // rows beyond this take the tensor-core path (faster from M = 5 on)
 constexpr uint32_t kStageWBytes = kStageRows * kTileV * 2;  // 32 KB
 constexpr uint32_t kStageZBytes = kStageRows * kZPad * 2;   // 1 KB
@@ -46,6 +46,10 @@ struct Plan {
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Phase-1 CTAs resident per SM (the kernel's launch bounds): the split-K grid
+// is sized to one wave of them, so no partial second wave trails the stream.
+__host__ __device__ constexpr int w1_blocks_per_sm(int M) { return M <= 2 ? 4 : 3; }
+
 inline int vocab_smem_bytes(int M, int nstages) {
   // stages + mbarriers + cross-warp reduction + reduced logits + 1 KB alignment slack
   return nstages * int(kStageWBytes + kStageZBytes) + 2 * nstages * 8 + kConsumerWarps * M * kTileV * 4 +
@@ -58,7 +62,9 @@ inline Plan make_plan(int M, int d, int V, int K, int kmax, int num_sms) {
   p.ntile_o = (d + kW1TileO - 1) / kW1TileO;
   int splits = 1;
   while (d / splits > kW1MaxRows) splits *= 2;
-  while (p.ntile_o * K * splits < 4 * num_sms && d / (splits * 2) >= 64 && (d / (splits * 2)) % 8 == 0) splits *= 2;
+  const int w1_slots = w1_blocks_per_sm(M) * num_sms;
+  while (p.ntile_o * K * splits * 2 <= w1_slots && d / (splits * 2) >= 64 && (d / (splits * 2)) % 8 == 0)
+    splits *= 2;
   p.splits = splits;
   p.rows = d / splits;
   p.ntiles = (V + kTileV - 1) / kTileV;
@@ -96,7 +102,7 @@ struct W1Args {
 };
 
 template <int M>
-__global__ void __launch_bounds__(kW1Threads) heads_w1_kernel(W1Args a) {
+__global__ void __launch_bounds__(kW1Threads, w1_blocks_per_sm(M)) heads_w1_kernel(W1Args a) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint4* hs = reinterpret_cast<uint4*>(smem);                          // [rows] x 8 bf16
   float* red = reinterpret_cast<float*>(smem + size_t(a.rows) * 16);   // [8 warps][M][256]
