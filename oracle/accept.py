@@ -21,6 +21,19 @@ row and its entropy ``H = -sum p ln p``, child j matches iff
 ``p(tokens[j]) > min(eps, alpha * exp(-H))`` (strict, natural log). Same path
 rule; the bonus token is still the greedy argmax. This rule is parity
 unpinned against the pages: only its limiting cases are fixed.
+
+Sampled (lossless) rule (same section: "if exactness matters, use standard
+rejection sampling"; the page gives no algorithm for a tree of deterministic
+candidates). Reading: rejection sampling of a candidate chosen with certainty
+(a point-mass draft q = delta_c) accepts it with probability p(c) and, on
+rejection, samples from p with c removed; over the candidate children of a node
+in turn this is the same as drawing one token y from p = softmax(logits /
+temperature) of the node's row and accepting the child whose token is y. So
+each row t gets one draw ``y_t = min{v : sum_{w <= v} p(w) > u_t}`` (inverse
+CDF in id order) from a supplied uniform u_t in [0, 1); node j matches iff
+``tokens[j] == y[parent(j)]``; same path rule; the bonus token is y of the last
+accepted node. The emitted tokens then follow the target's own sampling
+distribution exactly (pinned by simulation in the tests).
 """
 from __future__ import annotations
 
@@ -126,3 +139,37 @@ def typical_accept(logits, tokens, parent, K: int, temperature: float, eps: floa
 
 def tree_depth(parent) -> int:
     return int(depths(parent).max())
+
+
+def inverse_cdf_sample(row, temperature: float, u: float):
+    """One draw from p = softmax(row / temperature) (fp64): the smallest id v
+    with sum_{w <= v} p(w) > u; if rounding leaves u at or above the total, the
+    last id with p > 0. Returns (v, margin), margin = the distance from u to
+    the nearer end of v's CDF interval (how far the decision is from a tie)."""
+    p, _ = typical_stats(row, temperature)
+    cdf = np.cumsum(p)
+    v = int(np.searchsorted(cdf, u, side="right"))
+    if v >= len(p):
+        v = int(np.flatnonzero(p > 0)[-1])
+    lo = cdf[v - 1] if v > 0 else 0.0
+    return v, float(min(u - lo, cdf[v] - u))
+
+
+def sampled_accept(logits, tokens, parent, K: int, temperature: float, uniforms):
+    """Sampled acceptance. Returns (accept_len [B], path [B, K+1], bonus [B],
+    y [B, T] (each row's draw), margin [B, T])."""
+    B, T, _ = logits.shape
+    y = np.zeros((B, T), dtype=np.int64)
+    margin = np.zeros((B, T))
+    acc_len = np.zeros(B, dtype=np.int32)
+    path = np.full((B, K + 1), -1, dtype=np.int32)
+    bonus = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        for t in range(T):
+            y[b, t], margin[b, t] = inverse_cdf_sample(logits[b, t], temperature, float(uniforms[b, t]))
+        match = [False] + [int(tokens[b, j]) == int(y[b, parent[j]]) for j in range(1, T)]
+        L, pth = _walk_paths(match, parent, K)
+        acc_len[b] = L
+        path[b, :L + 1] = pth
+        bonus[b] = y[b, pth[-1]]
+    return acc_len, path, bonus, y, margin

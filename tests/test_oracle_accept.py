@@ -170,3 +170,62 @@ def test_typical_stats_two_level_row():
     q = 1 / (e + V - 1)
     assert abs(p[6] - p1) < 1e-15 and abs(p[0] - q) < 1e-15
     assert abs(H - (-p1 * math.log(p1) - (V - 1) * q * math.log(q))) < 1e-13
+
+
+# ------------------------- sampled (lossless) acceptance -------------------------
+
+def test_inverse_cdf_on_exact_rows():
+    """Rows whose probabilities are exact binary fractions: the draw is the
+    smallest id whose CDF exceeds u, ids with zero probability are never drawn
+    and a draw of u exactly on a boundary goes to the next id."""
+    row = np.zeros(4)                                   # p = 1/4 each, CDF .25 .5 .75 1
+    for u, v in [(0.0, 0), (0.2499, 0), (0.25, 1), (0.5, 2), (0.7499, 2), (0.75, 3), (0.99999, 3)]:
+        assert oacc.inverse_cdf_sample(row, 1.0, u)[0] == v, u
+    row = np.array([0.0, -np.inf, 0.0, 0.0])            # p = 1/3, 0, 1/3, 1/3
+    assert [oacc.inverse_cdf_sample(row, 1.0, u)[0] for u in (0.1, 0.34, 0.7)] == [0, 2, 3]
+    # temperature divides the logits: logits (0, 2 ln 3) at temperature 2 give p = (1/4, 3/4)
+    row = np.array([0.0, 2 * math.log(3.0)])
+    assert oacc.inverse_cdf_sample(row, 2.0, 0.249)[0] == 0
+    assert oacc.inverse_cdf_sample(row, 2.0, 0.251)[0] == 1
+
+
+def test_sampled_acceptance_reproduces_the_target_distribution():
+    """Rejection sampling must leave the target's sampling distribution intact:
+    over many uniform draws, the first emitted token (the accepted child's
+    token, else the bonus) follows the root row's softmax, and the token after
+    an accepted child follows that child's row."""
+    V = 5
+    parent = np.array([-1, 0, 0, 1])                    # root -> {1, 2}; 1 -> {3}
+    tokens = np.array([[0, 1, 3, 2]])
+    rng = np.random.default_rng(7)
+    logits = rng.normal(0.0, 1.0, (1, 4, V))
+    tau = 0.8
+    N = 20000
+    u = rng.random((N, 4))
+    first, second_after_1 = [], []
+    for i in range(N):
+        L, path, bonus, y, _ = oacc.sampled_accept(logits, tokens, parent, 2, tau, u[i][None, :])
+        emitted = [int(tokens[0, j]) for j in path[0, 1:L[0] + 1]] + [int(bonus[0])]
+        first.append(emitted[0])
+        if emitted[0] == 1:
+            second_after_1.append(emitted[1])
+    for counts, row in ((np.bincount(first, minlength=V), logits[0, 0]),
+                        (np.bincount(second_after_1, minlength=V), logits[0, 1])):
+        p, _ = oacc.typical_stats(row, tau)
+        n = counts.sum()
+        sigma = np.sqrt(n * p * (1 - p))
+        assert np.all(np.abs(counts - n * p) <= 5 * sigma + 1), (counts, n * p)
+
+
+def test_sampled_acceptance_tends_to_greedy_at_low_temperature():
+    """With well-separated logits and a temperature near zero every draw is the
+    argmax, so the sampled rule accepts exactly what the greedy rule accepts."""
+    kph, n = (4, 3, 2, 2), 16
+    parent, _, _ = ot.spec_from_tuples(ot.select_tree(kph, TREE_ACCEPT, n))
+    tokens = synth.synthetic_tree_tokens(3, 4, parent, 64)
+    logits = synth.planted_logits(3, parent, tokens, 64, TREE_ACCEPT, bump=4.0)
+    g = oacc.greedy_accept(logits, tokens, parent, 4)
+    u = np.random.default_rng(1).random((4, len(parent)))
+    s = oacc.sampled_accept(logits, tokens, parent, 4, 1e-3, u)
+    for i in range(3):
+        assert np.array_equal(g[i], s[i])
