@@ -56,12 +56,18 @@ HEADS_SOURCES = ("heads.cuh", "common.cuh")
 
 
 def heads_source_digest() -> str:
+    """sha256 (first 16 hex digits) of the heads sources with comments and
+    whitespace removed: a change of code invalidates a recorded capture, a
+    change of wording does not."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in HEADS_SOURCES:
-        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "medusa_draft_heads_b200", "csrc", f),
-                  "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "medusa_draft_heads_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", "", src).encode())
     return h.hexdigest()[:16]
 
 
@@ -332,6 +338,8 @@ def run_medusa(args, w):
     step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
                       Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
                       alpha=w.alpha, device=dev, shared_vocab=w.shared_vocab)
+    if step.uniforms is not None:      # sampled acceptance: seeded uniforms, one per tree row
+        step.uniforms.copy_(torch.rand(step.uniforms.shape, generator=torch.Generator().manual_seed(w.seed)))
     head_row = None
     if w.M != w.B:
         head_row = torch.arange(w.B, dtype=torch.int32, device=dev) * w.T
@@ -513,6 +521,8 @@ def run_part(args, w):
     step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
                       Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
                       alpha=w.alpha, device=dev, shared_vocab=w.shared_vocab)
+    if step.uniforms is not None:      # sampled acceptance: seeded uniforms, one per tree row
+        step.uniforms.copy_(torch.rand(step.uniforms.shape, generator=torch.Generator().manual_seed(w.seed)))
     P = synth.prefix_lengths(seed, w.B, *w.prefix)
     prefix = torch.from_numpy(P).to(dev)
     if args.part == "heads":
@@ -688,6 +698,8 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
         "v_new": torch.stack([vc0[b, :, Pn[b]:Pn[b] + w.T].cpu() for b in range(w.B)]).pin_memory(),
         "logits": lg0.cpu().pin_memory(),
     }
+    if step.uniforms is not None:      # sampled acceptance draws from per-step uniforms
+        host["uniforms"] = step.uniforms.cpu().pin_memory()
     out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
                 (("accept_len", step.accept_len), ("path", step.path), ("bonus", step.bonus))}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -707,6 +719,8 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
                 kc0[b, :, Pn[b]:Pn[b] + w.T].copy_(host["k_new"][b], non_blocking=True)
                 vc0[b, :, Pn[b]:Pn[b] + w.T].copy_(host["v_new"][b], non_blocking=True)
             lg0.copy_(host["logits"], non_blocking=True)
+            if step.uniforms is not None:
+                step.uniforms.copy_(host["uniforms"], non_blocking=True)
             copied.record(copy_stream)
         h.copy_(host["h"], non_blocking=True)
         root.copy_(host["root"], non_blocking=True)

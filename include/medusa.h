@@ -4,13 +4,13 @@
  *
  * The step, as "Medusa heads versus separate draft model" describes it
  * (sections "What each one is" and "Acceptance", tree paragraph):
- *   1. K draft heads read the target's last hidden state once, in parallel;
- *      head k is one residual block followed by its own vocabulary
- *      projection and guesses the token k positions ahead;
- *   2. the top few candidates of each head are combined into a tree;
- *   3. the target verifies every branch in one pass with a tree attention
+ *   1. K draft heads read the target's last hidden state in a single
+ *      parallel pass; head k applies a residual block and then a vocabulary
+ *      projection of its own, drafting the token k places ahead;
+ *   2. the heads' best-scoring candidates, combined, make up a tree;
+ *   3. the target checks every branch at once under a tree-shaped attention
  *      mask;
- *   4. the step advances along the longest branch that matches.
+ *   4. decoding continues along the longest matching branch.
  * Calls: md_medusa_heads (1), md_tree_build (2), md_tree_attention (3, one
  * attention layer of the verification pass), md_tree_accept (4).
  *
@@ -91,8 +91,8 @@ typedef struct md_tree md_tree;
 
 /* Creates a tree spec.
  * Source: "Medusa heads versus separate draft model", section "Acceptance",
- * tree paragraph ("take the top few candidates from each head, form a tree
- * of combinations").
+ * tree paragraph (each head offers its best-scoring candidates and their
+ * combinations make up the tree).
  *
  * Node 0 is the root (the token the target already emitted). A node at
  * depth k >= 1 is a candidate from head k: it holds head_rank[j], the rank
@@ -122,9 +122,10 @@ MD_API md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, 
 
 /* The K Medusa heads on M hidden rows, fused with a top-k per head.
  * Source: "Medusa heads versus separate draft model", sections "What each
- * one is" (one residual block and its own vocabulary projection per head,
- * all heads on the same hidden state, run once in parallel) and "Cost per
- * step" (block d x d + bias; projection d x V, no bias).
+ * one is" (per head a residual block, then a vocabulary projection of its
+ * own; all heads read the same hidden state in one parallel pass) and "Cost
+ * per step" (a d x d layer with bias in the block; a bias-free d x V
+ * projection).
  *
  *   u[m,k,o]      = b1[k,o] + sum_i h[m,i] * W1[k,i,o]          (fp32 accumulate)
  *   z[m,k,o]      = bf16_rne( h[m,o] + u / (1 + exp(-u)) )        (SiLU residual)
@@ -153,7 +154,7 @@ MD_API md_status md_heads_shared_workspace(int32_t M, int32_t d, int32_t V, int3
  * Source: "Medusa heads versus separate draft model", section "What
  * interviewers probe next": each head normally has its own d x V projection
  * (initialised from the LM head); sharing one saves (K - 1) d V parameters
- * (3.15B for four heads at d = 8,192, V = 128,256) at some cost to
+ * (3.15B of them for four heads at d = 8,192, V = 128,256) and costs some
  * acceptance. The residual blocks stay per head:
  *   z[m,k,:]     = bf16_rne( h[m,:] + SiLU(h[m,:] W1[k] + b1[k]) )
  *   logit[m,k,v] = sum_i z[m,k,i] * Wv[i,v]
@@ -236,8 +237,8 @@ MD_API md_status md_attention_workspace(int32_t B, int32_t T, int32_t Hq, int32_
 
 /* Attention of the T tree tokens over the KV prefix plus the tree.
  * Source: "Medusa heads versus separate draft model", section "Acceptance",
- * tree paragraph ("verify all branches in one pass with a tree attention
- * mask").
+ * tree paragraph (every branch is checked in a single target pass under a
+ * tree-shaped attention mask).
  *
  *   out[b,t,h,:] = sum_j softmax_j( scale * q[b,t,h,:] . K[b,g,j,:] ) V[b,g,j,:]
  *   over key slots j in [0, P_b) and P_b + a for every ancestor a of t
@@ -266,7 +267,7 @@ MD_API md_status md_accept_workspace(int32_t B, int32_t T, int32_t V, size_t* by
 
 /* Longest accepted root-to-node path per request, and the bonus token.
  * Source: "Medusa heads versus separate draft model", section "Acceptance",
- * tree paragraph ("if any branch matches, the step advances along it"), and
+ * tree paragraph (decoding continues along the branch that matches), and
  * section "Training" (typical acceptance: accepts more drafts, not lossless).
  *
  * Row t of logits is the target's distribution for the token after node t.
@@ -289,13 +290,41 @@ MD_API md_status md_tree_accept(const float* logits, int32_t V, const int32_t* t
                          int32_t* accept_len, int32_t* path, int32_t* bonus, void* ws, size_t ws_bytes,
                          void* stream);
 
+
+/* Sampled (lossless) acceptance: the emitted tokens follow the target's own
+ * sampling distribution.
+ * Source: "Medusa heads versus separate draft model", section "Training" (when
+ * the target distribution must be kept exactly, the page recommends rejection
+ * sampling instead of typical acceptance); it gives no algorithm for a tree of
+ * deterministic top-k candidates. Reading: rejection sampling of a candidate chosen with
+ * certainty (a point-mass draft) accepts it with probability p(c) and else
+ * samples p with c removed; over a node's candidate children this is one draw
+ * y_t ~ p_t of the node's row, accepting the child whose token is y_t.
+ *
+ *   p_t = softmax(logits[b,t,:] / temperature)
+ *   y_t = min{ v : sum_{w <= v} p_t(w) > uniforms[b,t] }   (ids in order)
+ *   non-root node j passes iff tokens[b,j] == y_{parent(j)}; the path rule is
+ *   md_tree_accept's; bonus[b] = y of the last accepted node.
+ *
+ * uniforms [B, T] fp32 in [0, 1), device: the random numbers are the caller's
+ *          (one per tree row), so runs are reproducible.
+ * temperature > 0. V <= 2,097,152 and V % 8 == 0. Other arguments as for
+ * md_tree_accept; the workspace is md_accept_workspace's. Draws are made in
+ * fp32 with fixed summation order: a uniform within ~1e-5 (relative) of a CDF
+ * boundary may resolve to the neighbouring id compared with exact arithmetic.
+ * A token outside [0, V) never matches a draw.
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED, MD_ERR_WORKSPACE, MD_ERR_CUDA. */
+MD_API md_status md_tree_accept_sampled(const float* logits, int32_t V, const int32_t* tokens, const md_tree* tree,
+                                        int32_t B, int32_t K, float temperature, const float* uniforms,
+                                        int32_t* accept_len, int32_t* path, int32_t* bonus, void* ws,
+                                        size_t ws_bytes, void* stream);
 /* ------------------------------------------------------------------------ */
 /* 5. Advancing along the accepted branch.                                   */
 /* ------------------------------------------------------------------------ */
 
 /* KV compaction and the next step's inputs, after md_tree_accept.
  * Source: "Medusa heads versus separate draft model", section "Acceptance",
- * tree paragraph ("if any branch matches, the step advances along it").
+ * tree paragraph (decoding continues along the branch that matches).
  *
  * For request b with P = prefix_len[b], L = accept_len[b], path = path[b]:
  *   K/V slot P + i  <-  K/V slot P + path[i]      (i = 0..L, in place; other

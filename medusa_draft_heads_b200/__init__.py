@@ -5,6 +5,7 @@
     tree_build     candidate tree: tokens, parents, ancestor bitsets, positions
     tree_attention tree-masked GQA attention over the KV prefix plus the tree
     tree_accept    longest accepted branch (greedy or typical) and bonus token
+    tree_accept_sampled  the same under lossless sampling (one draw per row)
     tree_commit    advance along it: KV compaction and the next step's inputs
 
 The kernels live in ``libmedusa.so`` (built from ``csrc/`` for sm_100a); this
@@ -12,6 +13,6 @@ package only marshals arguments to it.
 """
 from .binding import (MedusaError, Tree, accept_workspace_bytes, attention_workspace_bytes,  # noqa: F401
                       device_status, heads_shared_workspace_bytes, heads_workspace_bytes, lib, medusa_heads,
-                      medusa_heads_shared, tree_accept, tree_attention,
+                      medusa_heads_shared, tree_accept, tree_accept_sampled, tree_attention,
                       tree_build, tree_commit, version, workspace)
 from .tree_spec import select_tree, tree_arrays  # noqa: F401

@@ -39,6 +39,7 @@ _SIGNATURES = {
     "md_tree_attention": [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P],
     "md_accept_workspace": [_I, _I, _I, ctypes.POINTER(_SZ)],
     "md_tree_accept": [_P, _I, _P, _P, _I, _I, _I, _F, _F, _F, _P, _P, _P, _P, _SZ, _P],
+    "md_tree_accept_sampled": [_P, _I, _P, _P, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "md_tree_commit": [_P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
     "md_get_device_status": [_P, ctypes.POINTER(_I), _I],
     "md_status_string": [_I],
@@ -252,6 +253,23 @@ def tree_accept(logits, tokens, tree: Tree, accept_len, path, bonus, ws, mode="g
         _ptr(path, torch.int32, "path", 2), _ptr(bonus, torch.int32, "bonus"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream))
     _check(rc, "md_tree_accept")
+
+
+def tree_accept_sampled(logits, tokens, tree: Tree, uniforms, accept_len, path, bonus, ws, temperature=1.0,
+                        stream=None):
+    """md_tree_accept_sampled: logits [B,T,V] fp32, tokens [B,T], uniforms [B,T] fp32 in [0, 1)
+    -> accept_len [B], path [B,K+1], bonus [B] (lossless sampled acceptance)."""
+    B, T, V = logits.shape
+    K = path.shape[1] - 1
+    _same("tree_accept_sampled", T=(T, tree.T), tokens=(tuple(tokens.shape), (B, T)),
+          uniforms=(tuple(uniforms.shape), (B, T)), accept_len=(tuple(accept_len.shape), (B,)),
+          bonus=(tuple(bonus.shape), (B,)), path_rows=(path.shape[0], B))
+    rc = lib().md_tree_accept_sampled(
+        _ptr(logits, torch.float32, "logits", 3), V, _ptr(tokens, torch.int32, "tokens", 2), tree.handle, B, K,
+        float(temperature), _ptr(uniforms, torch.float32, "uniforms", 2), _ptr(accept_len, torch.int32, "accept_len"),
+        _ptr(path, torch.int32, "path", 2), _ptr(bonus, torch.int32, "bonus"), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream))
+    _check(rc, "md_tree_accept_sampled")
 
 
 def tree_commit(k_cache, v_cache, tree: Tree, prefix_len, accept_len, path, bonus, new_prefix_len, next_root,

@@ -13,6 +13,17 @@
 //                       its parent's row, propagate acceptance down the tree
 //                       level by level, pick the deepest accepted node (lowest
 //                       index on ties), emit its path and the bonus token.
+//   accept_sample_kernel (sampled rule) one draw per row by inverse CDF from a
+//                       supplied uniform; the walk then tests each node against
+//                       its parent's draw instead of the argmax.
+//
+// Sampled rule (same section: rejection sampling is the page's choice when the
+// target distribution must be kept exactly; it gives no algorithm for a tree
+// of deterministic candidates):
+// rejection sampling of a candidate chosen with certainty accepts it with
+// probability p(c) and otherwise samples p with c removed, which over a node's
+// candidate children is one draw y ~ p of the node's row, accepting the child
+// whose token is y; the bonus token is the last accepted node's draw.
 #pragma once
 
 #include "common.cuh"
@@ -30,6 +41,7 @@ struct Args {
   int32_t* path;           // [B, K + 1]
   int32_t* bonus;          // [B]
   float* part;             // [B * T, nchunks, 8]
+  const int32_t* ysamp;    // [B * T] per-row draws (sampled rule), else null
   int T, V, K, nchunks, chunk_len, mode;
   float inv_temp, log_eps, log_alpha;
 };
@@ -162,7 +174,9 @@ __global__ void __launch_bounds__(MD_MAX_T) accept_walk_kernel(const __grid_cons
   __shared__ int wkey[MD_MAX_T / 32];
   const bool typical = a.mode == MD_ACCEPT_TYPICAL;
 
-  if (j < T) {
+  if (j < T && a.ysamp) {
+    amax[j] = a.ysamp[size_t(b) * T + j];
+  } else if (j < T) {
     const float* p = a.part + size_t(b * T + j) * a.nchunks * kPartFloats;
     float bv = p[0];
     int bi = __float_as_int(p[1]);
@@ -222,6 +236,141 @@ __global__ void __launch_bounds__(MD_MAX_T) accept_walk_kernel(const __grid_cons
       pp[i] = node;
       node = tp.parent[node];
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Sampled rule: y = min{v : sum_{w <= v} p(w) > u} for p = softmax(x / temp) of
+// one row, in id order. One CTA per row: each warp takes 1024-id tiles and
+// records the tile maximum and sum of exp(x - max) (fixed order); one thread
+// combines the tiles in id order and finds the tile where u * S is crossed;
+// warp 0 then walks that tile's ids in order (lane l owns ids 32l .. 32l+31).
+// Rounding can leave the crossing just past the end of the tile or of the row:
+// then the last id with nonzero weight there is taken.
+// ---------------------------------------------------------------------------
+constexpr int kSampleTile = 1024;
+constexpr int kSampleMaxTiles = 2048;       // V <= 2M
+constexpr int kSampleThreads = 1024;        // 32 warps share a row's tiles: one row per CTA
+
+struct SampleArgs {
+  const float* logits;     // [B * T, V]
+  const float* uniforms;   // [B * T] in [0, 1)
+  int32_t* ysamp;          // [B * T]
+  int V;
+  float inv_temp_log2e;    // log2(e) / temperature
+};
+
+__global__ void __launch_bounds__(kSampleThreads) accept_sample_kernel(SampleArgs a) {
+  pdl_wait_primary();          // logits may come from earlier kernels
+  pdl_launch_dependents();
+  __shared__ float tmax[kSampleMaxTiles], tsum[kSampleMaxTiles];
+  __shared__ int s_tile;
+  __shared__ float s_rem, s_max;
+  const int row = blockIdx.x;
+  const float* x = a.logits + size_t(row) * a.V;
+  const int ntile = (a.V + kSampleTile - 1) / kSampleTile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float c = a.inv_temp_log2e;          // work in log2 units: y = x * log2(e) / temp
+  // pass 1: tile maxima and sums, one warp per tile
+  for (int i = warp; i < ntile; i += kSampleThreads / 32) {
+    float v[32];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int id = i * kSampleTile + j * 128 + lane * 4;
+      float4 f = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (id + 3 < a.V) {
+        f = ld_stream_f4(x + id);
+      } else {
+        if (id < a.V) f.x = x[id];
+        if (id + 1 < a.V) f.y = x[id + 1];
+        if (id + 2 < a.V) f.z = x[id + 2];
+      }
+      v[4 * j] = f.x * c;
+      v[4 * j + 1] = f.y * c;
+      v[4 * j + 2] = f.z * c;
+      v[4 * j + 3] = f.w * c;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx = fmaxf(mx, v[4 * j + e]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float sm = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) sm += exp2f(v[k] - mx);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
+    if (lane == 0) {
+      tmax[i] = mx;
+      tsum[i] = sm;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int i = 0; i < ntile; ++i) M = fmaxf(M, tmax[i]);
+    float S = 0.f;
+    for (int i = 0; i < ntile; ++i) S += (tmax[i] == -INFINITY) ? 0.f : tsum[i] * exp2f(tmax[i] - M);
+    const float target = a.uniforms[row] * S;
+    float C = 0.f;
+    int found = -1, last = -1;
+    float rem = INFINITY;
+    for (int i = 0; i < ntile; ++i) {
+      const float w = (tmax[i] == -INFINITY) ? 0.f : tsum[i] * exp2f(tmax[i] - M);
+      if (w > 0.f) last = i;
+      if (found < 0 && C + w > target) {
+        found = i;
+        rem = target - C;
+      }
+      C += w;
+    }
+    if (found < 0) found = last;             // rounding left u * S at the end: last tile with weight
+    s_tile = found;
+    s_rem = rem;
+    s_max = M;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int i = s_tile;
+    int y = 0;
+    if (i >= 0) {
+      const float M = s_max, rem = s_rem;
+      float w[32];
+      float ls = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int id = i * kSampleTile + lane * 32 + e;
+        w[e] = id < a.V ? exp2f(x[id] * c - M) : 0.f;
+        ls += w[e];
+      }
+      float incl = ls;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      const float excl = incl - ls;
+      const unsigned hit = __ballot_sync(0xffffffffu, ls > 0.f && rem < incl);
+      const unsigned pos = __ballot_sync(0xffffffffu, ls > 0.f);
+      // the first lane whose running sum passes rem, else the last lane with weight
+      const int src = hit ? __ffs(hit) - 1 : (pos ? 31 - __clz(pos) : 0);
+      int yl = -1, lastpos = -1;
+      if (lane == src) {
+        float run = excl;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          run += w[e];
+          if (w[e] > 0.f) lastpos = e;
+          if (yl < 0 && w[e] > 0.f && run > rem) yl = e;
+        }
+        if (yl < 0) yl = lastpos;
+      }
+      yl = __shfl_sync(0xffffffffu, yl, src);
+      y = i * kSampleTile + src * 32 + max(yl, 0);
+    }
+    if (lane == 0) a.ysamp[row] = y;
   }
 }
 

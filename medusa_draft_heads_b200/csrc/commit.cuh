@@ -1,7 +1,7 @@
 // Advancing along the accepted branch: KV compaction and next-step handoff.
 //
 // Source: "Medusa heads versus separate draft model", section "Acceptance",
-// tree paragraph ("the step advances along it"). The accepted path's tokens
+// tree paragraph (decoding continues along the branch that matches). The accepted path's tokens
 // join the sequence, so their K/V move next to the prefix: slot P + i receives
 // slot P + path[i] (i = 0..L). Moves are tiny (at most K + 1 rows per KV head)
 // and latency-bound: one CTA per (KV head, request) stages the source rows in

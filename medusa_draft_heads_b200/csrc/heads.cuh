@@ -1,11 +1,11 @@
 // Medusa draft heads with a fused per-head top-k, small-M streaming path.
 //
 // Source: "Medusa heads versus separate draft model", sections "What each one
-// is" and "Cost per step": head k = one residual block (d x d + bias) and its
-// own d x V vocabulary projection (no bias), all heads on the same hidden
-// state, once per step. At small batch the heads are bound by the bytes of
-// their weights (8.94 GB for four heads at d = 8,192, V = 128,256), so both
-// phases stream the weights once from HBM with 16-byte or TMA loads and do the
+// is" and "Cost per step": head k = a residual block around a d x d layer with
+// bias, then a bias-free d x V vocabulary projection of its own; all heads read
+// the same hidden state, once per step. At small batch the heads are bound by
+// the bytes of their weights (8.94 GB of them for four heads at d = 8,192,
+// V = 128,256), so both phases stream the weights once from HBM with 16-byte or TMA loads and do the
 // arithmetic in fp32 on the CUDA cores.
 //
 //   phase 1  heads_w1_kernel       u = h W1_k + b1_k, z_k = bf16(h + SiLU(u))

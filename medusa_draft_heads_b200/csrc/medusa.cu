@@ -872,6 +872,7 @@ md_status md_tree_accept(const float* logits, int32_t V, const int32_t* tokens, 
   md::acc::Args a;
   a.logits = logits; a.tokens = tokens; a.accept_len = accept_len; a.path = path; a.bonus = bonus;
   a.part = static_cast<float*>(ws);
+  a.ysamp = nullptr;
   a.T = T; a.V = V; a.K = K; a.nchunks = pl.nchunks; a.chunk_len = pl.chunk_len; a.mode = mode;
   a.inv_temp = mode == MD_ACCEPT_TYPICAL ? 1.0f / temperature : 1.0f;
   a.log_eps = std::log(eps);
@@ -880,6 +881,38 @@ md_status md_tree_accept(const float* logits, int32_t V, const int32_t* tokens, 
   if ((s = launch_pdl(md::acc::accept_rows_kernel, dim3(pl.nchunks, B * T), dim3(md::acc::kRowThreads), 0, st, a)) !=
       MD_OK)
     return s;
+  return launch_pdl(md::acc::accept_walk_kernel, dim3(B), dim3(MD_MAX_T), 0, st, tree->tp, a);
+}
+
+md_status md_tree_accept_sampled(const float* logits, int32_t V, const int32_t* tokens, const md_tree* tree,
+                                 int32_t B, int32_t K, float temperature, const float* uniforms,
+                                 int32_t* accept_len, int32_t* path, int32_t* bonus, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!logits || !tokens || !tree || !uniforms || !accept_len || !path || !bonus) return MD_ERR_INVALID_ARG;
+  const int T = tree->tp.T;
+  size_t need = 0;
+  md_status s = md_accept_workspace(B, T, V, &need);
+  if (s != MD_OK) return s;
+  if (V > md::acc::kSampleTile * md::acc::kSampleMaxTiles) return MD_ERR_UNSUPPORTED;
+  if (K < tree->tp.max_depth || K < 0) return MD_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !std::isfinite(temperature)) return MD_ERR_INVALID_ARG;
+  if (!aligned(logits, 16)) return MD_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the per-row draws take the front of the workspace (B*T ints <= its size)
+  int32_t* ysamp = static_cast<int32_t*>(ws);
+  md::acc::SampleArgs sa;
+  sa.logits = logits; sa.uniforms = uniforms; sa.ysamp = ysamp; sa.V = V;
+  sa.inv_temp_log2e = 1.4426950408889634f / temperature;
+  if ((s = launch_pdl(md::acc::accept_sample_kernel, dim3(B * T), dim3(md::acc::kSampleThreads), 0, st, sa)) !=
+      MD_OK)
+    return s;
+  md::acc::Args a;
+  a.logits = logits; a.tokens = tokens; a.accept_len = accept_len; a.path = path; a.bonus = bonus;
+  a.part = nullptr;
+  a.ysamp = ysamp;
+  a.T = T; a.V = V; a.K = K; a.nchunks = 0; a.chunk_len = 0; a.mode = MD_ACCEPT_GREEDY;
+  a.inv_temp = 1.0f; a.log_eps = 0.f; a.log_alpha = 0.f;
   return launch_pdl(md::acc::accept_walk_kernel, dim3(B), dim3(MD_MAX_T), 0, st, tree->tp, a);
 }
 

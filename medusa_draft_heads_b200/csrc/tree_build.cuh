@@ -1,8 +1,8 @@
 // Candidate tree construction.
 //
 // Source: "Medusa heads versus separate draft model", section "Acceptance",
-// tree paragraph: the top few candidates of each head are combined into a
-// tree. Node j at depth d takes the rank head_rank[j] candidate of head d.
+// tree paragraph: the heads' best-scoring candidates, combined across heads,
+// make up the tree. Node j at depth d takes the rank head_rank[j] candidate of head d.
 // Latency-bound (a few KB); one CTA per request, one thread per node.
 #pragma once
 

@@ -9,8 +9,8 @@ from __future__ import annotations
 import torch
 
 from .binding import (Tree, accept_workspace_bytes, attention_workspace_bytes, heads_shared_workspace_bytes,
-                      heads_workspace_bytes, medusa_heads, medusa_heads_shared, tree_accept, tree_attention,
-                      tree_build, tree_commit, workspace)
+                      heads_workspace_bytes, medusa_heads, medusa_heads_shared, tree_accept, tree_accept_sampled,
+                      tree_attention, tree_build, tree_commit, workspace)
 from .tree_spec import tree_arrays
 
 
@@ -43,6 +43,8 @@ class MedusaStep:
         self.next_root = torch.empty((B,), **i32)
         self.next_head_row = torch.empty((B,), **i32)
         self.shared_vocab = shared_vocab
+        # mode "sample": one uniform in [0, 1) per tree row, supplied by the caller
+        self.uniforms = torch.full((B, self.T), 0.5, **f32) if mode == "sample" else None
         ws_fn = heads_shared_workspace_bytes if shared_vocab else heads_workspace_bytes
         self.ws_heads = workspace(ws_fn(M, d, V, K, self.kmax), dev)
         self.ws_attn = workspace(attention_workspace_bytes(B, self.T, Hq, Hkv, dh, S_max), dev)
@@ -60,7 +62,15 @@ class MedusaStep:
     def attention(self, q, k_cache, v_cache, prefix_len, stream=None):
         tree_attention(q, k_cache, v_cache, prefix_len, self.tree, self.attn_out, self.ws_attn, stream=stream)
 
-    def accept(self, logits, stream=None):
+    def accept(self, logits, stream=None, uniforms=None):
+        """Greedy / typical acceptance, or (mode "sample") the lossless sampled
+        rule with one uniform per tree row ([B, T] fp32: `uniforms`, else the
+        step's own `self.uniforms`, which the caller refills each step)."""
+        if self.mode == "sample":
+            u = self.uniforms if uniforms is None else uniforms
+            tree_accept_sampled(logits, self.tokens, self.tree, u, self.accept_len, self.path, self.bonus,
+                                self.ws_acc, temperature=self.temperature, stream=stream)
+            return
         tree_accept(logits, self.tokens, self.tree, self.accept_len, self.path, self.bonus, self.ws_acc,
                     mode=self.mode, temperature=self.temperature, eps=self.eps, alpha=self.alpha, stream=stream)
 

@@ -10,16 +10,17 @@ nothing from the product path; the two share only ``seeded_inputs``.
 Sources (page title, then section):
 
 * "Medusa heads versus separate draft model", section "What each one is":
-  each head is one residual block on the target's last hidden state followed
-  by its own vocabulary projection; head k guesses the token k positions
-  ahead; all heads run once, in parallel.
-* same page, "Cost per step": residual block d x d + bias, vocabulary
-  projection d x V (no bias), d = 8,192, V = 128,256.
-* same page, "Acceptance": the tree paragraph (top few candidates per head,
-  a tree of their combinations, one verification pass with a tree attention
-  mask, advance along a matching branch) and the expected-length formula.
-* same page, "Training": typical acceptance, which accepts more drafts and is
-  not lossless.
+  a head is a residual block applied to the target's last hidden state,
+  then a vocabulary projection of its own; head k drafts the token k places
+  ahead, and the heads all read the same state in a single parallel pass.
+* same page, "Cost per step": a d x d layer with bias inside the block, a
+  bias-free d x V projection, d = 8,192, V = 128,256.
+* same page, "Acceptance": the tree paragraph (the heads' best candidates are
+  combined into a tree, the target checks all branches in a single masked
+  pass, decoding follows the branch that matches) and the expected-length
+  formula.
+* same page, "Training": typical acceptance (more drafts accepted, the target
+  distribution not kept) and rejection sampling when it must be kept.
 
 Pinning: every function here is pinned by ``tests/test_oracle_*.py`` against
 closed forms, brute force or printed values; the typical-acceptance rule is

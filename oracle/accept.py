@@ -1,8 +1,8 @@
 """Oracle: acceptance of the longest matching branch (test infrastructure).
 
 Definition followed ("Medusa heads versus separate draft model", section
-"Acceptance", tree paragraph): the tree is verified in one pass and, if any
-branch matches, the step advances along it. Row t of the target logits is the
+"Acceptance", tree paragraph): the target checks the whole tree in a single
+pass, and decoding continues along a branch that matches. Row t of the target logits is the
 target's distribution for the token after node t, so a non-root node j matches
 when its token is what the target emits after its parent.
 
@@ -14,17 +14,16 @@ L is the largest such count; the accepted path ends at the depth-L node with
 the smallest node index. The bonus token is the argmax of the last accepted
 node's row (the root's row when L = 0).
 
-Typical rule (same page, section "Training": typical acceptance accepts more
-drafts and does not preserve the target distribution; the page gives no
-formula). Reading: with ``p = softmax(logits / temperature)`` of the parent's
+Typical rule (same page, section "Training": typical acceptance trades the
+target distribution for more accepted drafts; the page gives no formula). Reading: with ``p = softmax(logits / temperature)`` of the parent's
 row and its entropy ``H = -sum p ln p``, child j matches iff
 ``p(tokens[j]) > min(eps, alpha * exp(-H))`` (strict, natural log). Same path
 rule; the bonus token is still the greedy argmax. This rule is parity
 unpinned against the pages: only its limiting cases are fixed.
 
-Sampled (lossless) rule (same section: "if exactness matters, use standard
-rejection sampling"; the page gives no algorithm for a tree of deterministic
-candidates). Reading: rejection sampling of a candidate chosen with certainty
+Sampled (lossless) rule (same section: the page recommends rejection sampling
+when the target distribution must be kept exactly, and gives no algorithm for a
+tree of deterministic candidates). Reading: rejection sampling of a candidate chosen with certainty
 (a point-mass draft q = delta_c) accepts it with probability p(c) and, on
 rejection, samples from p with c removed; over the candidate children of a node
 in turn this is the same as drawing one token y from p = softmax(logits /

@@ -1,8 +1,8 @@
 """Oracle: advancing along the accepted branch (test infrastructure).
 
 Definition followed ("Medusa heads versus separate draft model", section
-"Acceptance", tree paragraph): if a branch matches, the step advances along
-it. Reading: the tokens of the accepted path (root, then the L accepted
+"Acceptance", tree paragraph): decoding continues along the branch that
+matches. Reading: the tokens of the accepted path (root, then the L accepted
 nodes) join the sequence, so their keys and values must sit contiguously
 after the prefix; the bonus token becomes the next step's root; the next
 heads read the hidden state of the last accepted node.

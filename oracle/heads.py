@@ -1,12 +1,13 @@
 """Oracle: the K Medusa draft heads and the per-head top-k (test infrastructure).
 
 Definition followed ("Medusa heads versus separate draft model", sections
-"What each one is" and "Cost per step"): head k is one residual block on the
-target's last hidden state h, followed by its own d x V vocabulary projection.
+"What each one is" and "Cost per step"): head k applies a residual block
+to the target's last hidden state h and then a d x V vocabulary projection of
+its own.
 The block is read as ``z_k = h + SiLU(h W1_k + b1_k)`` (a d x d layer plus a
 bias: 67.1M parameters at d = 8,192); the projection has no bias (1,050.7M =
-d x V exactly). Head k predicts the token k positions ahead, and all heads read
-the same h ("run once, in parallel").
+d x V exactly). Head k drafts the token k places ahead, and every head reads the
+same h in a single parallel pass.
 
 Readings where the pages are silent:
 

@@ -1,8 +1,8 @@
 """Oracle: the candidate tree (test infrastructure).
 
 Definition followed ("Medusa heads versus separate draft model", section
-"Acceptance", tree paragraph): take the top few candidates of each head and
-form a tree of their combinations; head k guesses independently of heads
+"Acceptance", tree paragraph): each head offers its best-scoring candidates and
+their combinations make up the tree; head k guesses independently of heads
 1..k-1 ("What each one is"), so a node at depth k is a tuple of ranks
 (r_1, ..., r_k), and its token is the rank-r_k candidate of head k.
 

@@ -121,3 +121,79 @@ def test_bad_token_sets_status():
     acc, _, _ = _run(logits, tokens, parent, rank, 1, mode="typical")
     assert md.device_status(clear=True) == md.binding.DEV_BAD_TOKEN
     assert acc[0] == 0
+
+
+# ------------------------- sampled (lossless) acceptance -------------------------
+
+def _run_sampled(logits, tokens, parent, rank, K, u, temperature):
+    """Returns the outputs and the per-row draws (the library keeps them at the
+    front of the workspace, one int32 per tree row)."""
+    B, T, V = logits.shape
+    tree = md.Tree(parent, rank, [16] * K)
+    acc = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    path = torch.full((B, K + 1), -9, dtype=torch.int32, device="cuda")
+    bonus = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    ws = md.workspace(md.accept_workspace_bytes(B, T, V))
+    md.tree_accept_sampled(f32(logits), i32(tokens), tree, f32(u), acc, path, bonus, ws, temperature=temperature)
+    torch.cuda.synchronize()
+    y = ws[:B * T * 4].view(torch.int32).cpu().numpy().reshape(B, T)
+    return acc.cpu().numpy(), path.cpu().numpy(), bonus.cpu().numpy(), y
+
+
+@pytest.mark.parametrize("name,kph,n,B,V,sigma,bump,tau", [
+    ("tiny", (4, 3, 2, 2), 16, 4, 1024, 1.0, 2.0, 0.7),
+    ("70b-vocab", (10, 10, 10, 10), 64, 3, 128256, 3.0, 6.0, 0.7),
+    ("ragged-vocab", (10, 10, 10, 10), 16, 3, 5000, 3.0, 3.0, 1.0),
+])
+def test_sampled_matches_oracle(name, kph, n, B, V, sigma, bump, tau):
+    """Each row's draw equals the oracle's exact inverse-CDF draw wherever the
+    uniform is more than 1e-4 from a CDF boundary (elsewhere it must be one of
+    the ids whose interval is within 1e-4 of u); the walk over the GPU's draws
+    reproduces accept_len, path and bonus bit for bit."""
+    tups = ot.select_tree(kph, TREE_ACCEPT, n)
+    parent, rank, _ = ot.spec_from_tuples(tups)
+    seed = len(name) * 5
+    tokens = synth.synthetic_tree_tokens(seed, B, parent, V)
+    logits = synth.planted_logits(seed, parent, tokens, V, TREE_ACCEPT, sigma=sigma, bump=bump)
+    u = np.random.default_rng(seed).random((B, len(parent))).astype(np.float32)
+    acc, path, bonus, y = _run_sampled(logits, tokens, parent, rank, 4, u, tau)
+    racc, rpath, rbonus, ry, rmargin = oacc.sampled_accept(logits, tokens, parent, 4, tau, u.astype(np.float64))
+    assert md.device_status() == 0
+    near = rmargin <= 1e-4
+    assert np.array_equal(y[~near], ry[~near])
+    for b, t in zip(*np.nonzero(near)):
+        p, _ = oacc.typical_stats(logits[b, t], tau)
+        cdf = np.cumsum(p)
+        v = int(y[b, t])
+        lo = cdf[v - 1] if v > 0 else 0.0
+        assert p[v] > 0 and lo - 1e-4 <= u[b, t] < cdf[v] + 1e-4
+    # the walk over the GPU's own draws
+    for b in range(B):
+        match = [False] + [int(tokens[b, j]) == int(y[b, parent[j]]) for j in range(1, len(parent))]
+        L, pth = oacc._walk_paths(match, parent, 4)
+        assert acc[b] == L and list(path[b, :L + 1]) == pth and np.all(path[b, L + 1:] == -1)
+        assert bonus[b] == y[b, pth[-1]]
+    if not near.any():
+        assert np.array_equal(acc, racc) and np.array_equal(path, rpath) and np.array_equal(bonus, rbonus)
+    assert acc.max() > 0
+
+
+def test_sampled_low_temperature_is_greedy_on_gpu():
+    tups = ot.select_tree((4, 3, 2, 2), TREE_ACCEPT, 16)
+    parent, rank, _ = ot.spec_from_tuples(tups)
+    V = 4096
+    tokens = synth.synthetic_tree_tokens(9, 5, parent, V)
+    logits = synth.planted_logits(9, parent, tokens, V, TREE_ACCEPT, bump=4.0)
+    u = np.random.default_rng(2).random((5, len(parent))).astype(np.float32)
+    acc, path, bonus, _ = _run_sampled(logits, tokens, parent, rank, 4, u, 1e-3)
+    racc, rpath, rbonus, _ = oacc.greedy_accept(logits, tokens, parent, 4)
+    assert np.array_equal(acc, racc) and np.array_equal(path, rpath) and np.array_equal(bonus, rbonus)
+
+
+def test_sampled_rejects_bad_temperature():
+    parent, rank = [-1, 0], [0, 0]
+    logits = np.zeros((1, 2, 256), dtype=np.float32)
+    tokens = np.array([[1, 2]], dtype=np.int32)
+    u = np.full((1, 2), 0.5, dtype=np.float32)
+    with pytest.raises(md.MedusaError):
+        _run_sampled(logits, tokens, parent, rank, 1, u, 0.0)
