@@ -24,13 +24,10 @@
 // Work split: as in heads_gemm.cuh, but per row PAIR: the grid is `groups`
 // row-pair tiles x per_mt pairs, pair j of every group taking the same
 // contiguous range of the K * ntiles (head, column tile) units, so the pairs
-// sharing a weight strip read it at the same time. Block order is (j, group,
-// CTA of the pair) and, when the groups fit one cluster (2 * groups <= 8), the
-// launch makes each j one cluster: the pairs that share strips then sit in one
-// GPC, on one die, and read each weight line through the same L2 within a
-// short window instead of pulling it into both dies' L2 at different times.
-// Within a cluster of 2 * groups CTAs the pair partner is the CTA whose
-// cluster rank differs in bit 0; the even one leads.
+// sharing a weight strip read it at about the same time. Block order is (j,
+// group, CTA of the pair). The kernel works in clusters of any even size (the
+// pair partner is the CTA whose cluster rank differs in bit 0; the even one
+// leads); the launcher uses clusters of two.
 #pragma once
 
 #include "heads_gemm.cuh"

@@ -176,7 +176,7 @@ struct GemmPlan {
   int mtiles, ntiles1, ntiles2;
   bool pair;              // CTA-pair kernel (M > 128)
   int groups;             // row tiles (single CTAs) or row-tile pairs (pairs)
-  int cluster;            // pair kernel: CTAs per cluster (2 * groups when <= 8, else 2)
+  int cluster;            // pair kernel: CTAs per cluster (2), else 0
   int per_mt1, per_mt2;   // CTAs (pairs) per group of the two GEMMs
   int grid1, grid2;
   size_t off_z, off_cval, off_cid, bytes;
@@ -227,13 +227,10 @@ GemmPlan gemm_plan(int M, int d, int V, int K, int kmax) {
   int slots = num_sms();
   p.cluster = 0;
   if (p.pair) {
+    // one cluster per pair: clusters of all the row-pair groups of a unit range
+    // (one GPC) measured slower, with fewer resident CTAs and no fewer HBM reads
     p.cluster = 2;
-    int nc = pair_max_clusters(p.cluster);
-    if (nc <= 0 && p.cluster > 2) {
-      p.cluster = 2;
-      nc = pair_max_clusters(2);
-    }
-    slots = std::max(1, nc) * p.cluster / 2;   // resident pairs
+    slots = std::max(1, pair_max_clusters(p.cluster));   // resident pairs
   }
   p.per_mt1 = gemm_per_mt(slots, p.groups, K * p.ntiles1);
   p.per_mt2 = gemm_per_mt(slots, p.groups, K * p.ntiles2);
