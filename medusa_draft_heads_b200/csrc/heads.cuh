@@ -460,12 +460,13 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 // up to kmax entries. In "partitioned" mode slot c is CTA c of the kernel that
 // produced them (the CTAs that worked on row m): that kernel split `units`
 // work units, ordered (head, column tile of `ntiles`), into contiguous CTA
-// ranges, and only CTAs whose range touches head k wrote a list. The lists
-// that were written are compacted into shared memory (kk entries each, empty
-// entries as (-inf, INT_MAX)), padded to a power of two and bitonic-sorted in
-// the top-k order (value descending, then id ascending); the first kk entries
-// are the head's top-k. A few hundred candidates: ~40 shallow stages instead
-// of kk dependent rounds of warp arg-max.
+// ranges, and only CTAs whose range touches head k wrote a list. Every list
+// is sorted and holds kk entries at or above its kk-th, so the head's top kk
+// lie at or above the best of the lists' kk-th entries: only entries at or
+// above that threshold (typically a few dozen of the few hundred) are
+// compacted into shared memory, padded to a power of two and bitonic-sorted in
+// the top-k order (value descending, then id ascending); the first kk are the
+// head's top-k.
 // ---------------------------------------------------------------------------
 struct MergeArgs {
   const float* cand_val;
@@ -519,29 +520,90 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
     }
     __syncthreads();
   }
-  const int n = n_lists * kk;
-  int N = 32;
-  while (N < n) N <<= 1;
-
-  // 2. gather (value, id) pairs; pad with (-inf, INT_MAX)
-  for (int e = threadIdx.x; e < N; e += kMergeThreads) {
-    float v = -INFINITY;
-    int id = INT_MAX;
-    if (e < n) {
-      const int c = slot_of[e / kk], j = e % kk;
-      const size_t at = base + size_t(c) * a.kmax + j;
+  // 2. a threshold: each list holds kk entries at or above its own kk-th, so
+  // the head's top kk all lie at or above the best of the lists' kk-th
+  // entries; only those entries are sorted.
+  __shared__ float red_v[kMergeThreads / 32];
+  __shared__ int red_i[kMergeThreads / 32];
+  __shared__ int n_keep;
+  {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    for (int l = threadIdx.x; l < n_lists; l += kMergeThreads) {
+      const size_t at = base + size_t(slot_of[l]) * a.kmax + (kk - 1);
       const int x = a.cand_id[at];
       if (x >= 0) {
-        v = a.cand_val[at];
-        id = x;
+        const float v = a.cand_val[at];
+        if (better(v, x, bv, bi)) {
+          bv = v;
+          bi = x;
+        }
       }
     }
-    sv[e] = v;
-    si[e] = id;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      red_v[warp] = bv;
+      red_i[warp] = bi;
+    }
+    if (threadIdx.x == 0) n_keep = 0;
+    __syncthreads();
+  }
+  float tv = red_v[0];
+  int ti = red_i[0];
+#pragma unroll
+  for (int w = 1; w < kMergeThreads / 32; ++w)
+    if (better(red_v[w], red_i[w], tv, ti)) {
+      tv = red_v[w];
+      ti = red_i[w];
+    }
+
+  // 3. gather the (value, id) pairs at or above the threshold, in slot order
+  const int n = n_lists * kk;
+  for (int e0 = 0; e0 < n; e0 += kMergeThreads) {
+    const int e = e0 + threadIdx.x;
+    float v = -INFINITY;
+    int id = -1;
+    if (e < n) {
+      const size_t at = base + size_t(slot_of[e / kk]) * a.kmax + e % kk;
+      id = a.cand_id[at];
+      if (id >= 0) v = a.cand_val[at];
+    }
+    const bool keep = id >= 0 && (better(v, id, tv, ti) || (v == tv && id == ti));
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int off = n_keep;
+    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
+    if (keep) {
+      sv[off + __popc(bal & ((1u << lane) - 1))] = v;
+      si[off + __popc(bal & ((1u << lane) - 1))] = id;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = n_keep;
+      for (int w = 0; w < kMergeThreads / 32; ++w) t += warp_cnt[w];
+      n_keep = t;
+    }
+    __syncthreads();
+  }
+  const int nk = n_keep;
+  int N = 32;
+  while (N < nk) N <<= 1;
+  for (int e = nk + threadIdx.x; e < N; e += kMergeThreads) {   // pad with (-inf, INT_MAX)
+    sv[e] = -INFINITY;
+    si[e] = INT_MAX;
   }
   __syncthreads();
 
-  // 3. bitonic sort, best first
+  // 4. bitonic sort, best first
   for (int size = 2; size <= N; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int t = threadIdx.x; t < (N >> 1); t += kMergeThreads) {
@@ -559,7 +621,7 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
     }
   }
 
-  // 4. the first kk entries; the rest of the kmax slots are empty
+  // 5. the first kk entries; the rest of the kmax slots are empty
   if (threadIdx.x < a.kmax) {
     const int r = threadIdx.x;
     const bool used = r < kk && r < N && si[r] != INT_MAX;
