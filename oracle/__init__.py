@@ -21,10 +21,13 @@ Sources (page title, then section):
   formula.
 * same page, "Training": typical acceptance (more drafts accepted, the target
   distribution not kept) and rejection sampling when it must be kept.
+* "Hydra: Sequentially-Dependent Draft Heads for Medusa Decoding" (abstract):
+  draft heads whose guesses are conditioned on the earlier tokens of the
+  candidate continuation (``hydra.py``; the architecture is a reading).
 
 Pinning: every function here is pinned by ``tests/test_oracle_*.py`` against
 closed forms, brute force or printed values; the typical-acceptance rule is
 "parity unpinned" against the pages (they name the rule without its formula),
 and is pinned only by its limiting cases.
 """
-from . import accept, attention, heads, tree  # noqa: F401
+from . import accept, attention, heads, hydra, tree  # noqa: F401

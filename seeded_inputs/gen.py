@@ -57,6 +57,7 @@ STREAMS = {
     "prefix_len": 11,
     "tokens": 12,
     "plant_pick": 13,
+    "E": 14,
 }
 
 _U64 = np.uint64
