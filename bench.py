@@ -55,6 +55,26 @@ TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "prof
 HEADS_SOURCES = ("heads.cuh", "common.cuh")
 
 
+def hydra_levels(parent):
+    """Nodes with children at each depth (per request): the head rows of
+    each level of md_hydra_draft."""
+    depth = [0] * len(parent)
+    for j in range(1, len(parent)):
+        depth[j] = depth[parent[j]] + 1
+    with_children = set(parent[1:])
+    return [sum(1 for p in with_children if depth[p] == lvl) for lvl in range(max(depth))]
+
+
+def hydra_bytes(w, levels):
+    """Per level: one head's weights, the h and E rows its inputs read, its top-k out."""
+    head = 2 * (w.d * w.d + w.d + w.d * w.V)
+    return sum(head + 2 * 2 * w.B * n * w.d + 8 * w.B * n * w.kmax for n in levels)
+
+
+def hydra_flops(w, levels):
+    return sum(2 * w.B * n * (w.d * w.d + w.d * w.V) for n in levels)
+
+
 def heads_source_digest() -> str:
     """sha256 (first 16 hex digits) of the heads sources with comments and
     whitespace removed: a change of code invalidates a recorded capture, a
@@ -533,6 +553,18 @@ def run_part(args, w):
         h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), seed, "h", 1.0)
         call = lambda i: step.heads(h, W1, b1, Wv)                              # noqa: E731
         nbytes, nflops, launches = heads_bytes(w), heads_flops(w), 3
+    elif args.part == "hydra":
+        W1 = sdev.fill_normal(torch.empty((w.K, w.d, w.d), **bf), seed, "W1", w.w_sigma)
+        b1 = sdev.fill_normal(torch.empty((w.K, w.d), **bf), seed, "b1", w.w_sigma)
+        Wv = sdev.fill_normal(torch.empty((w.K, w.d, w.V), **bf), seed, "Wv", w.w_sigma)
+        h = sdev.fill_normal(torch.empty((w.M, w.d), **bf), seed, "h", 1.0)
+        E = sdev.fill_normal(torch.empty((w.V, w.d), **bf), seed, "E", 1.0)
+        root = torch.from_numpy(synth.root_tokens(seed, w.B, w.V)).to(dev)
+        ws_h = md.workspace(md.hydra_workspace_bytes(step.tree, w.B, w.d, w.V, w.kmax), dev)
+        call = lambda i: md.hydra_draft(step.tree, h, E, W1, b1, Wv, root, prefix, step.tokens,  # noqa: E731
+                                        step.parent, step.anc, step.pos, ws_h)
+        levels = hydra_levels(step.tree.parent)
+        nbytes, nflops, launches = hydra_bytes(w, levels), hydra_flops(w, levels), 4 * len(levels) + 1
     elif args.part == "attention":
         nsets = 8
         sets = [(sdev.fill_normal(torch.empty((w.B, w.T, w.Hq, w.dh), **bf), seed + i, "q", 1.0),
@@ -778,7 +810,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["medusa", "reference"], default="medusa")
     ap.add_argument("--workload", default="llama3-70b", choices=sorted(WORKLOADS))
-    ap.add_argument("--part", choices=["step", "heads", "attention", "accept", "commit"], default="step",
+    ap.add_argument("--part", choices=["step", "heads", "hydra", "attention", "accept", "commit"], default="step",
                     help="time one call alone (profiling); the JSON line then reports that call only")
     ap.add_argument("--sweep", action="store_true",
                     help="run the 8B-shaped sweep (B x tree x prefix x rule), one JSON line per point")

@@ -229,6 +229,60 @@ MD_API md_status md_tree_build(const md_tree* tree, const int32_t* topk_ids, int
                         void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* 1+2 (sequentially dependent heads). Hydra drafting of the whole tree.     */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes md_hydra_draft needs for this tree and these sizes. */
+MD_API md_status md_hydra_workspace(const md_tree* tree, int32_t B, int32_t d, int32_t V, int32_t kmax,
+                                    size_t* bytes);
+
+/* Drafts every node of the tree with sequentially dependent heads, then
+ * writes the tree outputs of md_tree_build.
+ * Sources: "Medusa heads versus separate draft model", section "Acceptance"
+ * (a Medusa head drafts without knowing the earlier heads' guesses);
+ * "Hydra: Sequentially-Dependent Draft Heads for Medusa Decoding" (abstract:
+ * drop-in draft heads whose guesses are conditioned on the earlier tokens of
+ * the candidate continuation). The pages give no Hydra architecture; this
+ * call reads it as the Medusa head of md_medusa_heads applied to the hidden
+ * state plus the input embedding of the parent node's token:
+ *
+ *   x_p           = bf16_rne( h[row_b] + E[tokens[b,p]] )   (exact sum, one rounding)
+ *   head l        = the residual block and projection of md_medusa_heads with
+ *                   W1[l], b1[l], Wv[l], applied to x_p for every node p at
+ *                   depth l that has children, top-k_l fused;
+ *   tokens[b,j]   = entry head_rank[j] of that top-k of x_parent(j);
+ *   tokens[b,0]   = root_token[b]; parent, anc, pos as md_tree_build.
+ *
+ * The heads run depth by depth (depth l needs the tokens of depth l), each
+ * level on B * n_l rows (n_l = nodes at depth l with children).
+ *
+ * tree       the spec; K must equal the K it was created with.
+ * h          [M, d] bf16; row_b = head_row ? head_row[b] : b (head_row [B] or NULL).
+ * E          [V, d] bf16 input token embedding of the target.
+ * W1 [K, d, d], b1 [K, d], Wv [K, d, V] bf16 as md_medusa_heads; h, E, W1,
+ *            b1 and Wv 16-byte aligned.
+ * kmax       >= every k of the tree's k_per_head.
+ * root_token [B], prefix_len [B] int32.
+ * tokens [B, T], parent [T], anc [T, W] uint32, pos [B, T] (outputs).
+ * logits_dbg NULL, or fp32 [rows, V] with rows = B * (n_0 + ... + n_{L-1}):
+ *            when given, the logits of every head row are also written
+ *            (debug / parity only), level by level, within a level request
+ *            by request, within a request the depth-l nodes with children
+ *            in node order.
+ * ws, ws_bytes: workspace of at least md_hydra_workspace() bytes, 256-byte aligned.
+ * A head_row outside [0, M) sets MD_DEV_BAD_ROW (that request's head inputs
+ * use a zero hidden state); a drafted token outside [0, V) sets
+ * MD_DEV_BAD_TOKEN (its embedding counts as zero).
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED (sizes md_medusa_heads does
+ * not take for one head on B * n_l rows), MD_ERR_WORKSPACE, MD_ERR_CUDA. */
+MD_API md_status md_hydra_draft(const md_tree* tree, const md_bf16* h, int32_t M, const int32_t* head_row,
+                                const md_bf16* E, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
+                                int32_t d, int32_t V, int32_t K, int32_t kmax, const int32_t* root_token,
+                                const int32_t* prefix_len, int32_t B, int32_t* tokens, int32_t* parent,
+                                uint32_t* anc, int32_t* pos, float* logits_dbg, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* 3. Tree-masked attention (one layer of the verification pass).            */
 /* ------------------------------------------------------------------------ */
 

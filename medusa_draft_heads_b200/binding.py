@@ -35,6 +35,9 @@ _SIGNATURES = {
     "md_heads_shared_workspace": [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
     "md_medusa_heads_shared": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
     "md_tree_build": [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
+    "md_hydra_workspace": [_P, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
+    "md_hydra_draft": [_P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _SZ,
+                       _P],
     "md_attention_workspace": [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
     "md_tree_attention": [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P],
     "md_accept_workspace": [_I, _I, _I, ctypes.POINTER(_SZ)],
@@ -222,6 +225,58 @@ def tree_build(tree: Tree, topk_ids, root_token, prefix_len, tokens, parent, anc
         _ptr(tokens, torch.int32, "tokens"), _ptr(parent, torch.int32, "parent"), _ptr(anc, torch.int32, "anc"),
         _ptr(pos, torch.int32, "pos"), _stream(stream))
     _check(rc, "md_tree_build")
+
+
+def hydra_workspace_bytes(tree: Tree, B, d, V, kmax) -> int:
+    n = _SZ()
+    _check(lib().md_hydra_workspace(tree.handle, B, d, V, kmax, ctypes.byref(n)), "md_hydra_workspace")
+    return n.value
+
+
+def hydra_logit_rows(tree: Tree, B):
+    """Row of each (request b, node p with children) in md_hydra_draft's debug
+    logits: level by level, then request by request, then the level's nodes
+    with children in node order. Returns ({(b, p): row}, rows)."""
+    parents = sorted(set(tree.parent[1:]))
+    depth = [0] * tree.T
+    for j in range(1, tree.T):
+        depth[j] = depth[tree.parent[j]] + 1
+    rows, r = {}, 0
+    for lvl in range(tree.max_depth):
+        nodes = [p for p in parents if depth[p] == lvl]
+        for b in range(B):
+            for p in nodes:
+                rows[(b, p)] = r
+                r += 1
+    return rows, r
+
+
+def hydra_draft(tree: Tree, h, E, W1, b1, Wv, root_token, prefix_len, tokens, parent, anc, pos, ws, kmax=None,
+                head_row=None, logits_dbg=None, stream=None):
+    """md_hydra_draft: sequentially dependent heads on h [M,d] with the input
+    embedding E [V,d] and W1 [K,d,d], b1 [K,d], Wv [K,d,V] (bf16) -> tokens
+    [B,T], parent [T], anc [T,W] (int32 view of uint32), pos [B,T]."""
+    M, d = h.shape
+    K, _, V = Wv.shape
+    kmax = max(tree.k_per_head) if kmax is None else int(kmax)
+    B = root_token.shape[0]
+    T, W = tree.T, (tree.T + 31) // 32
+    _same("hydra_draft", heads=(K, tree.K), E=(tuple(E.shape), (V, d)), W1=(tuple(W1.shape), (K, d, d)),
+          b1=(tuple(b1.shape), (K, d)), prefix_len=(tuple(prefix_len.shape), (B,)),
+          tokens=(tuple(tokens.shape), (B, T)), parent=(tuple(parent.shape), (T,)), anc=(tuple(anc.shape), (T, W)),
+          pos=(tuple(pos.shape), (B, T)))
+    if head_row is not None:
+        _same("hydra_draft", head_row=(tuple(head_row.shape), (B,)))
+    if logits_dbg is not None:
+        _same("hydra_draft", logits_dbg=(tuple(logits_dbg.shape), (hydra_logit_rows(tree, B)[1], V)))
+    rc = lib().md_hydra_draft(
+        tree.handle, _ptr(h, torch.bfloat16, "h", 2), M, _ptr(head_row, torch.int32, "head_row"),
+        _ptr(E, torch.bfloat16, "E", 2), _ptr(W1, torch.bfloat16, "W1", 3), _ptr(b1, torch.bfloat16, "b1", 2),
+        _ptr(Wv, torch.bfloat16, "Wv", 3), d, V, K, kmax, _ptr(root_token, torch.int32, "root_token"),
+        _ptr(prefix_len, torch.int32, "prefix_len"), B, _ptr(tokens, torch.int32, "tokens"),
+        _ptr(parent, torch.int32, "parent"), _ptr(anc, torch.int32, "anc"), _ptr(pos, torch.int32, "pos"),
+        _ptr(logits_dbg, torch.float32, "logits_dbg", 2), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "md_hydra_draft")
 
 
 def tree_attention(q, k_cache, v_cache, prefix_len, tree: Tree, out, ws, scale=0.0, stream=None):

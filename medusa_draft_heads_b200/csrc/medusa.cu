@@ -17,6 +17,7 @@
 #include "attention_tc.cuh"
 #include "accept.cuh"
 #include "commit.cuh"
+#include "hydra.cuh"
 
 struct md_tree {
   md::TreeParams tp;
@@ -585,6 +586,60 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   return cuda_ok(cudaLaunchKernelEx(&cfg, attn_tc_kernel<DH>, qmap, kmap, vmap, tree->tp, a));
 }
 
+// ----------------------------- Hydra planning ------------------------------
+// Level l drafts the children of the depth-l nodes that have children: B * n[l]
+// head rows, top-k rows row0[l] + b * n[l] + slot[p] of one [rows, kmax] array.
+
+struct HydraPlan {
+  int L;                              // levels: the depth of the deepest node
+  int n[MD_MAX_K];                    // nodes with children at depth l (per request)
+  int row0[MD_MAX_K];                 // first top-k row of level l
+  int rows;                           // top-k rows of all levels
+  int8_t slot[MD_MAX_T];              // node -> index among its depth's nodes with children (-1: none)
+  int8_t node[MD_MAX_K][MD_MAX_T];    // level l, index q -> node
+  size_t heads_bytes;                 // largest heads workspace of one level
+  size_t off_x, off_ids, off_vals, off_heads, bytes;
+};
+
+md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPlan* out) {
+  using md::heads::align256;
+  const TreeParams& tp = tree->tp;
+  HydraPlan p;
+  std::memset(&p, 0, sizeof(p));
+  p.L = tp.max_depth;
+  bool has_child[MD_MAX_T] = {};
+  for (int j = 1; j < tp.T; ++j) has_child[tp.parent[j]] = true;
+  for (int j = 0; j < tp.T; ++j) {
+    p.slot[j] = -1;
+    if (!has_child[j]) continue;
+    const int l = tp.depth[j];
+    p.node[l][p.n[l]] = int8_t(j);
+    p.slot[j] = int8_t(p.n[l]++);
+  }
+  md_status s = heads_check(1, d, V, 1, kmax);
+  if (s != MD_OK) return s;
+  int rows = 0, maxn = 1;
+  p.heads_bytes = 0;
+  for (int l = 0; l < p.L; ++l) {
+    p.row0[l] = rows;
+    rows += B * p.n[l];
+    maxn = std::max(maxn, p.n[l]);
+    if (tree->kph[l] > kmax) return MD_ERR_INVALID_ARG;
+    size_t hb = 0;
+    if ((s = md_heads_workspace(B * p.n[l], d, V, 1, kmax, &hb)) != MD_OK) return s;
+    p.heads_bytes = std::max(p.heads_bytes, hb);
+  }
+  p.rows = rows;
+  size_t o = 0;
+  p.off_x = o;     o = align256(o + size_t(B) * maxn * d * 2);
+  p.off_ids = o;   o = align256(o + size_t(std::max(rows, 1)) * kmax * 4);
+  p.off_vals = o;  o = align256(o + size_t(std::max(rows, 1)) * kmax * 4);
+  p.off_heads = o; o = align256(o + p.heads_bytes);
+  p.bytes = o;
+  *out = p;
+  return MD_OK;
+}
+
 // Scratch of md_medusa_heads_static: a fixed array in the library's device
 // image (every GPU that loads the library holds it until the process exits).
 __device__ __align__(256) uint8_t g_heads_static_scratch[MD_HEADS_STATIC_SCRATCH_BYTES];
@@ -789,6 +844,75 @@ md_status md_tree_build(const md_tree* tree, const int32_t* topk_ids, int32_t M,
   a.M = M; a.K = tree->K; a.kmax = kmax;
   return launch_pdl(md::tree::tree_build_kernel, dim3(B), dim3(MD_MAX_T), 0, static_cast<cudaStream_t>(stream),
                     tree->tp, a);
+}
+
+md_status md_hydra_workspace(const md_tree* tree, int32_t B, int32_t d, int32_t V, int32_t kmax, size_t* bytes) {
+  if (!tree || !bytes || B < 1 || d < 1 || V < 1 || kmax < 1) return MD_ERR_INVALID_ARG;
+  HydraPlan p;
+  md_status s = hydra_plan(tree, B, d, V, kmax, &p);
+  if (s != MD_OK) return s;
+  *bytes = p.bytes;
+  return MD_OK;
+}
+
+md_status md_hydra_draft(const md_tree* tree, const md_bf16* h, int32_t M, const int32_t* head_row,
+                         const md_bf16* E, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, int32_t d,
+                         int32_t V, int32_t K, int32_t kmax, const int32_t* root_token, const int32_t* prefix_len,
+                         int32_t B, int32_t* tokens, int32_t* parent, uint32_t* anc, int32_t* pos,
+                         float* logits_dbg, void* ws, size_t ws_bytes, void* stream) {
+  if (!tree || !h || !E || !W1 || !b1 || !Wv || !root_token || !prefix_len || !tokens || !parent || !anc || !pos)
+    return MD_ERR_INVALID_ARG;
+  if (M < 1 || B < 1 || K != tree->K) return MD_ERR_INVALID_ARG;
+  if (!head_row && M < B) return MD_ERR_INVALID_ARG;
+  size_t need = 0;
+  md_status s = md_hydra_workspace(tree, B, d, V, kmax, &need);
+  if (s != MD_OK) return s;
+  if (!aligned(h, 16) || !aligned(E, 16) || !aligned(W1, 16) || !aligned(b1, 16) || !aligned(Wv, 16) ||
+      (logits_dbg && !aligned(logits_dbg, 4)))
+    return MD_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  HydraPlan p;
+  if ((s = hydra_plan(tree, B, d, V, kmax, &p)) != MD_OK) return s;
+  const TreeParams& tp = tree->tp;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* x = reinterpret_cast<uint16_t*>(w + p.off_x);
+  int32_t* ids = reinterpret_cast<int32_t*>(w + p.off_ids);
+  float* vals = reinterpret_cast<float*>(w + p.off_vals);
+  for (int l = 0; l < p.L; ++l) {
+    md::hydra::GatherArgs ga;
+    std::memset(&ga, 0, sizeof(ga));
+    ga.h = h; ga.E = E; ga.head_row = head_row; ga.root_token = root_token;
+    ga.prev_ids = l == 0 ? nullptr : ids + size_t(p.row0[l - 1]) * kmax;
+    ga.x = x;
+    ga.M = M; ga.d = d; ga.V = V; ga.kmax = kmax;
+    ga.n_prev = l == 0 ? 0 : p.n[l - 1];
+    for (int q = 0; q < p.n[l]; ++q) {
+      const int node = p.node[l][q];
+      ga.pslot[q] = l == 0 ? int8_t(0) : p.slot[tp.parent[node]];
+      ga.prank[q] = tp.rank[node];
+    }
+    if ((s = launch_pdl(md::hydra::hydra_gather_kernel, dim3(p.n[l], B), dim3(md::hydra::kGatherThreads), 0, st,
+                        ga)) != MD_OK)
+      return s;
+    const size_t r0 = size_t(p.row0[l]);
+    if ((s = md_medusa_heads(x, W1 + size_t(l) * d * d, b1 + size_t(l) * d, Wv + size_t(l) * d * V, B * p.n[l], d, V,
+                             1, &tree->kph[l], kmax, ids + r0 * kmax, vals + r0 * kmax,
+                             logits_dbg ? logits_dbg + r0 * V : nullptr, w + p.off_heads, p.heads_bytes, stream)) !=
+        MD_OK)
+      return s;
+  }
+  md::hydra::TokenArgs ta;
+  std::memset(&ta, 0, sizeof(ta));
+  ta.ids = ids; ta.root_token = root_token; ta.prefix_len = prefix_len;
+  ta.tokens = tokens; ta.parent = parent; ta.anc = anc; ta.pos = pos;
+  ta.kmax = kmax;
+  for (int l = 0; l < MD_MAX_K; ++l) {
+    ta.row0[l] = l < p.L ? p.row0[l] : 0;
+    ta.n[l] = l < p.L ? p.n[l] : 0;
+  }
+  for (int j = 0; j < MD_MAX_T; ++j) ta.slot[j] = p.slot[j];
+  return launch_pdl(md::hydra::hydra_tokens_kernel, dim3(B), dim3(MD_MAX_T), 0, st, tp, ta);
 }
 
 md_status md_attention_workspace(int32_t B, int32_t T, int32_t Hq, int32_t Hkv, int32_t dh, int32_t S_max,

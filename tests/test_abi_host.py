@@ -109,3 +109,66 @@ def test_product_tree_choice_equals_oracle(kph, a, n):
     parent, rank = tree_spec.tree_arrays(tree_spec.select_tree(kph, a, n))
     p2, r2, _ = ot.spec_from_tuples(ot.select_tree(kph, a, n))
     assert parent == list(p2) and rank[1:] == list(r2[1:])
+
+
+def _tree_handle(libmedusa, kph, n, accept=TREE_ACCEPT):
+    parent, rank = tree_spec.tree_arrays(tree_spec.select_tree(kph, accept, n))
+    h = ctypes.c_void_p()
+    assert libmedusa.md_tree_create(_i32(parent), _i32(rank), len(parent), len(kph), _i32(list(kph)),
+                                    ctypes.byref(h)) == 0
+    return h
+
+
+def test_hydra_workspace_queries(libmedusa):
+    n = ctypes.c_size_t()
+    h = _tree_handle(libmedusa, (10, 10, 10, 10), 64)
+    try:
+        assert libmedusa.md_hydra_workspace(h, 1, 8192, 128256, 10, ctypes.byref(n)) == 0
+        # at least the head inputs of the widest level (10 rows of d bf16) and
+        # the top-k ids and values of all 1 + 10 + 10 + 4 head rows
+        assert n.value >= 10 * 8192 * 2 + 2 * 25 * 10 * 4
+        one = n.value
+        assert libmedusa.md_hydra_workspace(h, 4, 8192, 128256, 10, ctypes.byref(n)) == 0 and n.value > one
+        assert libmedusa.md_hydra_workspace(h, 1, 100, 128256, 10, ctypes.byref(n)) == -2   # d % 64
+        assert libmedusa.md_hydra_workspace(h, 1, 8192, 128252, 10, ctypes.byref(n)) == -2  # V % 8
+        assert libmedusa.md_hydra_workspace(h, 1, 8192, 128256, 9, ctypes.byref(n)) == -1   # kmax < a head's k
+        assert libmedusa.md_hydra_workspace(h, 0, 8192, 128256, 10, ctypes.byref(n)) == -1
+        assert libmedusa.md_hydra_workspace(None, 1, 8192, 128256, 10, ctypes.byref(n)) == -1
+    finally:
+        libmedusa.md_tree_destroy(h)
+    root_only = ctypes.c_void_p()
+    assert libmedusa.md_tree_create(_i32([-1]), _i32([0]), 1, 1, _i32([1]), ctypes.byref(root_only)) == 0
+    try:
+        assert libmedusa.md_hydra_workspace(root_only, 2, 256, 1024, 1, ctypes.byref(n)) == 0 and n.value > 0
+    finally:
+        libmedusa.md_tree_destroy(root_only)
+
+
+def test_hydra_logit_rows_layout():
+    """Level by level, then request by request, then the level's nodes with
+    children in node order."""
+    import medusa_draft_heads_b200 as md
+    parent, rank = tree_spec.tree_arrays(tree_spec.select_tree((10, 10, 10, 10), TREE_ACCEPT, 64))
+    tree = md.Tree(parent, rank, (10, 10, 10, 10))
+    rows, total = md.hydra_logit_rows(tree, 2)
+    assert total == 2 * (1 + 10 + 10 + 4)
+    assert rows[(0, 0)] == 0 and rows[(1, 0)] == 1
+    assert [rows[(0, j)] for j in range(1, 11)] == list(range(2, 12))
+    assert [rows[(1, j)] for j in range(1, 11)] == list(range(12, 22))
+    with_children = sorted(set(parent[1:]))
+    assert sorted(rows) == sorted((b, p) for b in range(2) for p in with_children)
+    assert sorted(rows.values()) == list(range(total))
+
+
+def test_bench_hydra_level_accounting():
+    import bench
+    from seeded_inputs.workloads import LLAMA70B
+    # depths 0, 1, 1, 2, 2, 2, 3; nodes with children: 0 (depth 0), 1 and 2 (depth 1), 3 (depth 2)
+    assert bench.hydra_levels([-1, 0, 0, 1, 1, 2, 3]) == [1, 2, 1]
+    parent, _ = tree_spec.tree_arrays(tree_spec.select_tree((10, 10, 10, 10), TREE_ACCEPT, 64))
+    levels = bench.hydra_levels(parent)
+    assert levels == [1, 10, 10, 4]
+    w = LLAMA70B
+    # every level streams one head's weights once: the same weight bytes as the Medusa heads
+    weights = 4 * 2 * (w.d * w.d + w.d + w.d * w.V)
+    assert bench.hydra_bytes(w, levels) == weights + sum(4 * n * w.d + 8 * n * w.kmax for n in levels)
