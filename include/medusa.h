@@ -13,6 +13,7 @@
  *   4. decoding continues along the longest matching branch.
  * Calls: md_medusa_heads (1), md_tree_build (2), md_tree_attention (3, one
  * attention layer of the verification pass), md_tree_accept (4).
+ * md_hydra_draft does 1 and 2 with sequentially dependent (Hydra) heads.
  *
  * Conventions (all calls):
  *  - Tensor pointers are DEVICE pointers unless a comment says "host". The
@@ -65,7 +66,8 @@ enum {
 enum {
   MD_DEV_BAD_PREFIX = 1,   /* prefix_len[b] < 0 or prefix_len[b] + T > S_max     */
   MD_DEV_BAD_ROW = 2,      /* head_row[b] outside [0, M)                         */
-  MD_DEV_BAD_TOKEN = 4,    /* a token id outside [0, V) reached tree_accept      */
+  MD_DEV_BAD_TOKEN = 4,    /* a token id outside [0, V) reached tree_accept or   */
+                           /* a Hydra head input                                */
   MD_DEV_TIMEOUT = 8,      /* a pipeline wait exceeded its bound                 */
   MD_DEV_BAD_PATH = 16     /* md_tree_commit got a length or path that is not a  */
                            /* root-to-node path of the tree                       */
