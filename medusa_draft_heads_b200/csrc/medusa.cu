@@ -2,6 +2,7 @@
 //
 // One translation unit holds every kernel so that the device status word is a
 // single module-scope variable without relocatable device code.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -31,16 +32,18 @@ using md::TreeParams;
 
 constexpr int kMaxDevices = 64;
 
+// Host caches below are filled lazily and may be filled by several threads at
+// once; each writer stores the same value, and atomics make that well defined.
 int num_sms() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -61,14 +64,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -476,7 +482,8 @@ AcceptPlan accept_plan(int B, int T, int V) {
   const int max_chunks = (V + 1023) / 1024;
   // as many row chunks as fit one wave of resident CTAs (~4 per SM: enough
   // loads in flight), so that no second partial wave trails the scan
-  static int per_sm = 0;
+  static std::atomic<int> per_sm_cache{0};
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
   if (per_sm == 0) {
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, md::acc::accept_rows_kernel, md::acc::kRowThreads, 0) !=
@@ -486,6 +493,7 @@ AcceptPlan accept_plan(int B, int T, int V) {
       nb = 4;
     }
     per_sm = nb;
+    per_sm_cache.store(nb, std::memory_order_relaxed);
   }
   int n = per_sm * num_sms() / rows;
   n = std::max(1, std::min(n, max_chunks));
