@@ -143,3 +143,47 @@ def test_head_input_rounds_the_exact_sum_to_nearest_even():
     x = oh.bf16_to_f64(ohy.head_input(h, E, 0))
     # a tie goes to the even neighbour; above the tie rounds up; exact zero stays zero
     assert x.tolist() == [1.0, 1.0 + 2.0 ** -6, 1.0 + 2.0 ** -7, 0.0]
+
+
+def _random_tree(rng, T, kph):
+    """A tree of T nodes of any shape the library accepts: parent[j] < j,
+    depth <= len(kph), distinct ranks below one parent."""
+    parent, rank, depth = [-1], [0], [0]
+    used = {0: set()}
+    while len(parent) < T:
+        p = int(rng.integers(0, len(parent)))
+        if depth[p] >= len(kph):
+            continue
+        free = [r for r in range(kph[depth[p]]) if r not in used[p]]
+        if not free:
+            continue
+        r = int(rng.choice(free))
+        used[p].add(r)
+        used[len(parent)] = set()
+        parent.append(p)
+        rank.append(r)
+        depth.append(depth[p] + 1)
+    return np.array(parent), np.array(rank), np.array(depth)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_tree_shapes(seed):
+    """Trees not made by the tree selection (siblings out of rank order,
+    skipped ranks, uneven depths): the shift closed form and the reduction to
+    the Medusa tree both still hold."""
+    rng = np.random.default_rng(100 + seed)
+    kph = (5, 4, 3, 2)
+    parent, rank, depth = _random_tree(rng, 24, kph)
+    V = 64
+    h, E, W1, b1, Wv = _shift_weights(V, 4)
+    root = int(rng.integers(0, V))
+    tok, par, anc, pos, _ = ohy.hydra_draft(parent, rank, h, E, W1, b1, Wv, np.array([root]), np.array([3]))
+    assert np.array_equal(tok[0], _shift_expected(parent, rank, depth, root, V))
+    assert np.array_equal(pos[0], 3 + depth)
+    B, d, V2 = 1, 64, 256
+    hh, _, W1r, b1r, Wvr = _random_case(seed, B, d, V2)
+    Ez = np.zeros((V2, d), dtype=np.uint16)
+    t0, *_ = ohy.hydra_draft(parent, rank, hh, Ez, W1r, b1r, Wvr, np.array([7]), np.array([0]))
+    ids, _, _, _ = oh.medusa_heads(hh, W1r, b1r, Wvr, kph)
+    rtok, _, _, _ = ot.tree_build(parent, rank, ids, np.array([7]), np.array([0]))
+    assert np.array_equal(t0, rtok)
