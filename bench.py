@@ -47,7 +47,10 @@ L2_BYTES = 126 * 1024 * 1024
 # Algorithmic byte and flop counts (what the method must move / compute).
 # --------------------------------------------------------------------------- #
 def heads_bytes(w):
-    return w.head_weight_bytes() + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax
+    """Weights, hidden rows in, top-k out; sampled drafts also read one uniform
+    and write one logit per (row, head, token)."""
+    extra = 8 * w.M * w.K * w.V if w.mode == "rejection" else 0
+    return w.head_weight_bytes() + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax + extra
 
 
 TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
@@ -141,6 +144,11 @@ def attention_flops(w, P):
 
 
 def accept_bytes(w):
+    """Greedy / typical / sampled rules scan every tree row. The rejection rule
+    reads at most the K + 1 target rows on the accepted path and K head rows
+    per request (an upper bound: the walk stops at the first full rejection)."""
+    if w.mode == "rejection":
+        return w.B * (2 * w.K + 1) * w.V * 4
     return w.B * w.T * w.V * 4
 
 
@@ -307,9 +315,9 @@ def run_reference(args, w):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sec, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_dict(w, None),
-            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample},
+            "config": config_dict(w, synth.prefix_lengths(w.seed, w.B, *w.prefix)),
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(),
+                             "host_cpus": os.cpu_count(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -325,6 +333,17 @@ def config_dict(w, P):
 # --------------------------------------------------------------------------- #
 # The CUDA arm.
 # --------------------------------------------------------------------------- #
+def seed_step_uniforms(step, seed):
+    """Seeded uniforms for the rules that draw random numbers: one per tree row
+    (sampled acceptance), or per (row, head, token) for the draws plus two per
+    tree row for the tests and the bonus draw (rejection acceptance)."""
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    for t in (step.uniforms, step.u_draft, step.u_accept, step.u_residual):
+        if t is not None:
+            t.copy_(torch.rand(t.shape, generator=g).clamp_(1e-7, 1 - 1e-7))
+
+
 def run_medusa(args, w):
     import torch
     import torch.distributed as dist
@@ -358,8 +377,7 @@ def run_medusa(args, w):
     step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
                       Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
                       alpha=w.alpha, device=dev, shared_vocab=w.shared_vocab)
-    if step.uniforms is not None:      # sampled acceptance: seeded uniforms, one per tree row
-        step.uniforms.copy_(torch.rand(step.uniforms.shape, generator=torch.Generator().manual_seed(w.seed)))
+    seed_step_uniforms(step, w.seed)
     head_row = None
     if w.M != w.B:
         head_row = torch.arange(w.B, dtype=torch.int32, device=dev) * w.T
@@ -511,7 +529,8 @@ def run_medusa(args, w):
             "attention": {"bytes": ab, "flops": af, "gbs": ab / (attn_ms / 1000) / 1e9,
                           "tflops": af / (attn_ms / 1000) / 1e12},
             "accept": {"bytes": accept_bytes(w), "gbs": accept_bytes(w) / (acc_ms / 1000) / 1e9},
-            "gpu_launches": (3 + 1 + (1 if (128 % (w.Hq // w.Hkv)) == 0 else 2) + 2) * args.steps,
+            # heads 3, tree build 1, attention 2 (main + merge, or chunks + merge), acceptance 2 (1 rejection)
+            "gpu_launches": (3 + 1 + 2 + (1 if w.mode == "rejection" else 2)) * args.steps,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -541,8 +560,7 @@ def run_part(args, w):
     step = MedusaStep(B=w.B, M=w.M, d=w.d, V=w.V, K=w.K, k_per_head=w.k_per_head, tree_tuples=tups, Hq=w.Hq,
                       Hkv=w.Hkv, dh=w.dh, S_max=w.S_max, mode=w.mode, temperature=w.temperature, eps=w.eps,
                       alpha=w.alpha, device=dev, shared_vocab=w.shared_vocab)
-    if step.uniforms is not None:      # sampled acceptance: seeded uniforms, one per tree row
-        step.uniforms.copy_(torch.rand(step.uniforms.shape, generator=torch.Generator().manual_seed(w.seed)))
+    seed_step_uniforms(step, w.seed)
     P = synth.prefix_lengths(seed, w.B, *w.prefix)
     prefix = torch.from_numpy(P).to(dev)
     if args.part == "heads":
@@ -589,10 +607,12 @@ def run_part(args, w):
         logits = synth.planted_logits(seed, np.array(step.tree.parent), tokens, w.V, w.accept,
                                       sigma=w.logit_sigma, bump=w.bump)
         step.tokens.copy_(torch.from_numpy(tokens))
+        if step.logits_dbg is not None:    # rejection rule: the heads' logits (draft distributions)
+            sdev.fill_normal(step.logits_dbg, seed, "head_logits", 1.0)
         nsets = max(2, -(-2 * L2_BYTES // logits.nbytes))
         lgs = [torch.from_numpy(logits).to(dev) for _ in range(nsets)]
         call = lambda i: step.accept(lgs[i % nsets])                              # noqa: E731
-        nbytes, nflops, launches = accept_bytes(w), 0, 2
+        nbytes, nflops, launches = accept_bytes(w), 0, (1 if w.mode == "rejection" else 2)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             call(i)
@@ -730,13 +750,15 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
         "v_new": torch.stack([vc0[b, :, Pn[b]:Pn[b] + w.T].cpu() for b in range(w.B)]).pin_memory(),
         "logits": lg0.cpu().pin_memory(),
     }
-    if step.uniforms is not None:      # sampled acceptance draws from per-step uniforms
-        host["uniforms"] = step.uniforms.cpu().pin_memory()
+    # the rules that draw random numbers take this step's uniforms from the host
+    for name in ("uniforms", "u_draft", "u_accept", "u_residual"):
+        if getattr(step, name) is not None:
+            host[name] = getattr(step, name).cpu().pin_memory()
     out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
                 (("accept_len", step.accept_len), ("path", step.path), ("bonus", step.bonus))}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
-    steps = max(3, args.steps // 4)
+    steps = max(50, args.steps // 4)
 
     # The inputs the heads do not read (q, the tree K/V, the target logits:
     # nearly all of the bytes) are copied on a second stream while the heads
@@ -751,10 +773,13 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
                 kc0[b, :, Pn[b]:Pn[b] + w.T].copy_(host["k_new"][b], non_blocking=True)
                 vc0[b, :, Pn[b]:Pn[b] + w.T].copy_(host["v_new"][b], non_blocking=True)
             lg0.copy_(host["logits"], non_blocking=True)
-            if step.uniforms is not None:
-                step.uniforms.copy_(host["uniforms"], non_blocking=True)
+            for name in ("uniforms", "u_accept", "u_residual"):
+                if name in host:
+                    getattr(step, name).copy_(host[name], non_blocking=True)
             copied.record(copy_stream)
         h.copy_(host["h"], non_blocking=True)
+        if "u_draft" in host:          # the draws' uniforms feed the heads
+            step.u_draft.copy_(host["u_draft"], non_blocking=True)
         root.copy_(host["root"], non_blocking=True)
         prefix.copy_(host["prefix"], non_blocking=True)
         step.heads(h, W1, b1, Wv)
@@ -797,7 +822,8 @@ def cpu_baseline(w, args):
     while time.perf_counter() - t0 < args.cpu_seconds or len(est) < 2:
         est.append(smp.step())
     sec = float(np.median(est))
-    return {"value": 1.0 / sec, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+    return {"value": 1.0 / sec, "unit": "steps/s", "cores": blas_threads(), "host_cpus": os.cpu_count(),
+            "kind": "oracle",
             "sample": f"{len(est)} oracle sample steps in {time.perf_counter() - t0:.1f} s; each: residual block "
                       f"and vocabulary projection on {frac:.4g} of their output columns, attention on {frac:.4g} of "
                       f"its (token, head) rows, scaled by 1/{frac:.4g}; tree build and acceptance in full"}

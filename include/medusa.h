@@ -170,25 +170,59 @@ MD_API md_status md_medusa_heads_shared(const md_bf16* h, const md_bf16* W1, con
                                         float* topk_vals, float* logits_dbg, void* ws, size_t ws_bytes,
                                         void* stream);
 
+/* The draft heads with SAMPLED candidates: each head's k candidates are k
+ * draws without replacement from its own distribution
+ * q = softmax(logits / temperature), in draw order, instead of its top-k.
+ * Source: "Medusa heads versus separate draft model", section "Training"
+ * (rejection sampling keeps the target's distribution exactly; it needs drafts
+ * drawn from a known distribution, which md_tree_accept_rejection then uses).
+ *
+ * The draws use the Gumbel-top-k construction: with one caller-supplied
+ * uniform u in (0, 1) per (row, head, token),
+ *   key[m,k,v] = logit[m,k,v] / temperature - ln(-ln u[m,k,v]),
+ * and the candidates are the k_per_head[k] tokens of largest key, by key
+ * descending (ties to the lower id). The i-th candidate is then distributed as
+ * q restricted to the tokens not drawn before it. u = 0 or 1 gives a key of
+ * -inf or +inf.
+ *
+ *   uniforms   [M, K, V] fp32 (16-byte aligned), read once
+ *   topk_ids   [M, K, kmax] int32, the candidates in draw order (-1 padded)
+ *   topk_keys  [M, K, kmax] fp32, their keys (-inf padded)
+ *   logits     [M, K, V] fp32 (required, 16-byte aligned): the heads' logits,
+ *              which md_tree_accept_rejection reads as the draft distribution
+ * Everything else, the workspace (md_heads_workspace) and the errors are as
+ * md_medusa_heads; temperature must be positive and finite. */
+MD_API md_status md_medusa_heads_sampled(const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
+                                         const md_bf16* Wv, int32_t M, int32_t d, int32_t V, int32_t K,
+                                         const int32_t* k_per_head, int32_t kmax, float temperature,
+                                         const float* uniforms, int32_t* topk_ids, float* topk_keys, float* logits,
+                                         void* ws, size_t ws_bytes, void* stream);
+
 /* Size of the library-owned scratch behind md_medusa_heads_static (8 MiB). */
 #define MD_HEADS_STATIC_SCRATCH_BYTES (8u << 20)
 
 /* md_medusa_heads for callers that cannot allocate device memory.
  * (An addition of this library: the pages have no counterpart.)
  *
- * Some callers have no way to hand the library a workspace: code that runs
- * while a CUDA graph is being captured (where cudaMalloc is not allowed),
- * runtimes whose device memory is fully owned by a pool that no plugin may
- * grow, or hot loops that must never reach the allocator. This entry point
- * computes exactly what md_medusa_heads computes, with the same arguments
- * minus the workspace: its scratch is a fixed MD_HEADS_STATIC_SCRATCH_BYTES
- * array inside the library's device image, which every GPU that loads the
- * library keeps until the process exits. It calls no cudaMalloc, cudaFree or
- * other allocating routine. The caller still provides the inputs and outputs.
+ * Some callers have no way to hand the library a workspace: runtimes whose
+ * device memory is owned by a pool that no plugin may grow, or latency-bound
+ * decode loops that must never reach the allocator (cudaMalloc and cudaFree
+ * can synchronise the device and can fail for lack of memory at an
+ * unpredictable point). This entry point computes exactly what
+ * md_medusa_heads computes, with the same arguments minus the workspace: its
+ * scratch is a fixed MD_HEADS_STATIC_SCRATCH_BYTES array inside the
+ * library's device image, which every GPU that loads the library keeps until
+ * the process exits. It calls no cudaMalloc, cudaFree or other allocating
+ * routine. The caller still provides the inputs and outputs.
  *
- * - Sizes whose scratch (md_heads_workspace) exceeds the array are rejected
- *   with MD_ERR_WORKSPACE before anything is launched (at d = 8192,
- *   V = 128256, K = 4, kmax = 10 this admits M <= 74).
+ * - Arguments are checked as md_medusa_heads checks them first; then sizes
+ *   whose scratch (md_heads_workspace on the calling device) exceeds the
+ *   array are rejected with MD_ERR_WORKSPACE before anything is launched. The
+ *   scratch of the tensor-core path grows with the device's SM count, so the
+ *   largest admitted M depends on the GPU: on a 148-SM B200 at d = 8192,
+ *   V = 128256, K = 4, kmax = 10 it is M = 74. Callers that need a guarantee
+ *   compare md_heads_workspace(...) with MD_HEADS_STATIC_SCRATCH_BYTES on
+ *   their device.
  * - The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
  *   first call before any stream capture on the device.
@@ -374,6 +408,49 @@ MD_API md_status md_tree_accept_sampled(const float* logits, int32_t V, const in
                                         int32_t B, int32_t K, float temperature, const float* uniforms,
                                         int32_t* accept_len, int32_t* path, int32_t* bonus, void* ws,
                                         size_t ws_bytes, void* stream);
+
+/* Lossless acceptance of SAMPLED drafts (md_medusa_heads_sampled): rejection
+ * sampling against the heads' own distributions, so the emitted tokens follow
+ * the target's sampling distribution exactly.
+ * Source: "Medusa heads versus separate draft model", section "Training"
+ * (rejection sampling when the target distribution must be kept). The page
+ * gives no algorithm for a tree; reading (recursive rejection over the
+ * children of a node, drafts drawn without replacement):
+ *
+ *   At node t (root first) with target p = softmax(logits[b,t,:] / temperature)
+ *   and children c_1..c_m carrying head ranks 0..m-1 (tokens y_1..y_m, the
+ *   first m draws of head depth(t)), with that head's
+ *   q = softmax(head_logits[head_row[b], depth(t), :] / temperature_q):
+ *     r_1 = p; for i = 1..m: q_i = q without y_1..y_{i-1}, renormalised;
+ *       accept c_i iff u_accept[b,c_i] < r_i(y_i) / q_i(y_i);
+ *       else r_{i+1} = max(0, r_i - q_i) / sum max(0, r_i - q_i).
+ *   An accepted child's token is emitted and the walk continues there. If no
+ *   child is accepted, or t has no children, bonus[b] is drawn from r_{m+1}
+ *   (p at a leaf) by inverse CDF in id order with u_residual[b,t], and the
+ *   walk stops. accept_len[b] = accepted nodes; path[b] = root then the
+ *   accepted nodes, -1 padded to K + 1.
+ *
+ *   logits       [B, T, V] fp32 target logits, row t = after node t
+ *   tokens       [B, T] int32, from md_tree_build on md_medusa_heads_sampled's ids
+ *   head_logits  [M, Kh, V] fp32, md_medusa_heads_sampled's logits output
+ *   head_row     [B] int32 or NULL (request b uses row b): the heads row whose
+ *                draws built request b's tree
+ *   u_accept, u_residual  [B, T] fp32 uniforms in [0, 1), the caller's
+ *   temperature, temperature_q > 0: of the target and of the draft heads
+ * Every node's children must carry the ranks 0..m-1 (MD_ERR_UNSUPPORTED
+ * otherwise); K >= tree depth, Kh >= tree depth; V <= 196,608. One 8-CTA
+ * cluster per request; no workspace. Decisions are taken in fp32 with a fixed
+ * summation order: a uniform within ~1e-5 (relative) of its threshold or CDF
+ * boundary may resolve differently from exact arithmetic. A head row outside
+ * [0, M) (MD_DEV_BAD_ROW) accepts nothing; a token outside [0, V)
+ * (MD_DEV_BAD_TOKEN) is rejected.
+ * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED, MD_ERR_CUDA. */
+MD_API md_status md_tree_accept_rejection(const float* logits, int32_t V, const int32_t* tokens,
+                                          const md_tree* tree, int32_t B, int32_t K, float temperature,
+                                          const float* head_logits, int32_t M, int32_t Kh, const int32_t* head_row,
+                                          float temperature_q, const float* u_accept, const float* u_residual,
+                                          int32_t* accept_len, int32_t* path, int32_t* bonus, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* 5. Advancing along the accepted branch.                                   */
 /* ------------------------------------------------------------------------ */
@@ -410,6 +487,24 @@ MD_API md_status md_tree_commit(md_bf16* k_cache, md_bf16* v_cache, int32_t S_ma
 /* Synchronises `stream`, then stores the device status word (MD_DEV_* bits
  * set by kernels since the last clear) in *out; clears it if `clear` != 0. */
 MD_API md_status md_get_device_status(void* stream, int32_t* out, int32_t clear);
+
+/* Bound, in nanoseconds, on every pipeline wait of the library's kernels on
+ * the current device (0: the default, 2 s). A correct launch never comes near
+ * it; a wait that runs out flags MD_DEV_TIMEOUT and its kernel winds down and
+ * returns, leaving the context usable. Synchronous (a copy to device memory);
+ * affects kernels launched afterwards.
+ * Errors: MD_ERR_CUDA. */
+MD_API md_status md_set_wait_limit(uint64_t ns);
+
+/* Test hook for the timeout path (not for production use): while chunk >= 0,
+ * the producers of md_tree_attention's tensor-core kernel do not issue the K/V
+ * copies of that chunk (counted from 0 in each CTA's work range), so the waits
+ * that need them run out after md_set_wait_limit's bound: the call flags
+ * MD_DEV_TIMEOUT, every copy that was issued lands before its CTA exits, every
+ * tensor-core operation completes before TMEM is released, and the next call
+ * without the hook is correct. chunk = -1 turns it off. Synchronous.
+ * Errors: MD_ERR_INVALID_ARG (chunk < -1), MD_ERR_CUDA. */
+MD_API md_status md_test_withhold_attention_chunk(int32_t chunk);
 
 /* Static description of a status code. */
 MD_API const char* md_status_string(md_status status);

@@ -32,6 +32,7 @@ _SIGNATURES = {
     "md_tree_info": [_P, ctypes.POINTER(_I), ctypes.POINTER(_I)],
     "md_heads_workspace": [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
     "md_medusa_heads": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
+    "md_medusa_heads_sampled": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "md_heads_shared_workspace": [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)],
     "md_medusa_heads_shared": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
     "md_tree_build": [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
@@ -43,8 +44,11 @@ _SIGNATURES = {
     "md_accept_workspace": [_I, _I, _I, ctypes.POINTER(_SZ)],
     "md_tree_accept": [_P, _I, _P, _P, _I, _I, _I, _F, _F, _F, _P, _P, _P, _P, _SZ, _P],
     "md_tree_accept_sampled": [_P, _I, _P, _P, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
+    "md_tree_accept_rejection": [_P, _I, _P, _P, _I, _I, _F, _P, _I, _I, _P, _F, _P, _P, _P, _P, _P, _P],
     "md_tree_commit": [_P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
     "md_get_device_status": [_P, ctypes.POINTER(_I), _I],
+    "md_set_wait_limit": [ctypes.c_uint64],
+    "md_test_withhold_attention_chunk": [_I],
     "md_status_string": [_I],
     "md_version": [],
 }
@@ -188,6 +192,27 @@ def medusa_heads(h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, ws, logits_dbg=
     _check(rc, "md_medusa_heads")
 
 
+def medusa_heads_sampled(h, W1, b1, Wv, k_per_head, uniforms, topk_ids, topk_keys, logits, ws, temperature=1.0,
+                         stream=None):
+    """md_medusa_heads_sampled: the heads with candidates drawn from softmax(logits / temperature)
+    without replacement (Gumbel-top-k over uniforms [M,K,V] fp32) -> topk_ids [M,K,kmax] int32
+    (draw order), topk_keys [M,K,kmax] fp32, logits [M,K,V] fp32."""
+    M, d = h.shape
+    K, _, V = Wv.shape
+    kmax = topk_ids.shape[2]
+    _same("medusa_heads_sampled", W1=(tuple(W1.shape), (K, d, d)), b1=(tuple(b1.shape), (K, d)),
+          Wv=(tuple(Wv.shape), (K, d, V)), topk_ids=(tuple(topk_ids.shape), (M, K, kmax)),
+          topk_keys=(tuple(topk_keys.shape), (M, K, kmax)), k_per_head=(len(k_per_head), K),
+          uniforms=(tuple(uniforms.shape), (M, K, V)), logits=(tuple(logits.shape), (M, K, V)))
+    rc = lib().md_medusa_heads_sampled(
+        _ptr(h, torch.bfloat16, "h", 2), _ptr(W1, torch.bfloat16, "W1", 3), _ptr(b1, torch.bfloat16, "b1", 2),
+        _ptr(Wv, torch.bfloat16, "Wv", 3), M, d, V, K, _host_i32(k_per_head), kmax, float(temperature),
+        _ptr(uniforms, torch.float32, "uniforms", 3), _ptr(topk_ids, torch.int32, "topk_ids", 3),
+        _ptr(topk_keys, torch.float32, "topk_keys", 3), _ptr(logits, torch.float32, "logits", 3),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "md_medusa_heads_sampled")
+
+
 def medusa_heads_shared(h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, ws, logits_dbg=None, stream=None):
     """md_medusa_heads_shared: h [M,d], W1 [K,d,d], b1 [K,d], ONE Wv [d,V] bf16 ->
     topk_ids [M,K,kmax] int32, topk_vals [M,K,kmax] fp32."""
@@ -327,6 +352,28 @@ def tree_accept_sampled(logits, tokens, tree: Tree, uniforms, accept_len, path, 
     _check(rc, "md_tree_accept_sampled")
 
 
+def tree_accept_rejection(logits, tokens, tree: Tree, head_logits, u_accept, u_residual, accept_len, path, bonus,
+                          temperature=1.0, temperature_q=1.0, head_row=None, stream=None):
+    """md_tree_accept_rejection: lossless acceptance of sampled drafts. logits [B,T,V] fp32,
+    tokens [B,T], head_logits [M,Kh,V] fp32, u_accept / u_residual [B,T] fp32 in [0, 1)
+    -> accept_len [B], path [B,K+1], bonus [B]."""
+    B, T, V = logits.shape
+    M, Kh, Vh = head_logits.shape
+    K = path.shape[1] - 1
+    _same("tree_accept_rejection", T=(T, tree.T), tokens=(tuple(tokens.shape), (B, T)), head_V=(Vh, V),
+          u_accept=(tuple(u_accept.shape), (B, T)), u_residual=(tuple(u_residual.shape), (B, T)),
+          accept_len=(tuple(accept_len.shape), (B,)), bonus=(tuple(bonus.shape), (B,)), path_rows=(path.shape[0], B))
+    if head_row is not None:
+        _same("tree_accept_rejection", head_row=(tuple(head_row.shape), (B,)))
+    rc = lib().md_tree_accept_rejection(
+        _ptr(logits, torch.float32, "logits", 3), V, _ptr(tokens, torch.int32, "tokens", 2), tree.handle, B, K,
+        float(temperature), _ptr(head_logits, torch.float32, "head_logits", 3), M, Kh,
+        _ptr(head_row, torch.int32, "head_row"), float(temperature_q), _ptr(u_accept, torch.float32, "u_accept", 2),
+        _ptr(u_residual, torch.float32, "u_residual", 2), _ptr(accept_len, torch.int32, "accept_len"),
+        _ptr(path, torch.int32, "path", 2), _ptr(bonus, torch.int32, "bonus"), _stream(stream))
+    _check(rc, "md_tree_accept_rejection")
+
+
 def tree_commit(k_cache, v_cache, tree: Tree, prefix_len, accept_len, path, bonus, new_prefix_len, next_root,
                 next_head_row, stream=None):
     """md_tree_commit: move the accepted path's K/V next to the prefix (in place)
@@ -351,6 +398,16 @@ def device_status(clear: bool = True, stream=None) -> int:
     v = _I()
     _check(lib().md_get_device_status(_stream(stream), ctypes.byref(v), int(bool(clear))), "md_get_device_status")
     return v.value
+
+
+def set_wait_limit(ns: int = 0):
+    """md_set_wait_limit: bound (ns) on every pipeline wait; 0 restores the 2 s default."""
+    _check(lib().md_set_wait_limit(int(ns)), "md_set_wait_limit")
+
+
+def withhold_attention_chunk_for_test(chunk: int):
+    """md_test_withhold_attention_chunk: the timeout-path test hook (-1 = off)."""
+    _check(lib().md_test_withhold_attention_chunk(int(chunk)), "md_test_withhold_attention_chunk")
 
 
 def version() -> int:

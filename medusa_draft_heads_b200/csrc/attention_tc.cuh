@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + kSBufs;           // kSBufs
   uint64_t* o_full = p_full + kSBufs;           // 2: P_c V_c commits to o_full[c & 1]
   uint64_t* o_last = o_full + 2;                // 1: every P V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + 1);
+  uint64_t* mma_done = o_last + 1;              // 1: every MMA this CTA issued has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* req = reinterpret_cast<int*>(tmem_slot + 2);   // request served by this CTA
   float* xmax = reinterpret_cast<float*>(bars + 32);    // [2 halves][128 rows] chunk maxima
 
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&o_full[i]), 1);
     mbar_init(smem_u32(o_last), 1);
+    mbar_init(smem_u32(mma_done), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -199,7 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < C::KB; ++kb)
         tma_load_3d(smem_u32(sQ + kb * kBM * 128), &qmap, kb * 64, hk * a.G, b * T + rt * tpt, qb);
       bool ok = true;
+      int nk = 0, nv = 0;                    // chunks whose K / V copies were issued
+      const int withhold = *const_cast<volatile int*>(&g_withhold_chunk);   // test hook, normally -1
       for (int c = 0; c < nch && ok; ++c) {
+        if (c == withhold) continue;         // test hook: this chunk's copies never come
         const int st = c % kStages, ph = ((c / kStages) - 1) & 1;
         const int key0 = (c_begin + c) * kBN;
         uint8_t* sk = sKV + st * C::kStage;
@@ -209,19 +214,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(kb_, C::kKBytes);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(smem_u32(sk + kb * kBN * 128), &kmap, kb * 64, key0, kvrow, kb_);
+        nk = c + 1;
         if (c >= kStages && !mbar_wait(smem_u32(&v_empty[st]), ph)) { ok = false; break; }
         const uint32_t vb_ = smem_u32(&v_full[st]);
         mbar_arrive_expect_tx(vb_, C::kVBytes);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(smem_u32(sv + kb * kBN * 128), &vmap, kb * 64, key0, kvrow, vb_);
+        nv = c + 1;
       }
-      // drain: every issued copy has been consumed before the CTA can exit
-      for (int c = max(0, nch - kStages); c < nch && ok; ++c) {
-        if (!mbar_wait(smem_u32(&k_empty[c % kStages]), (c / kStages) & 1) ||
-            !mbar_wait(smem_u32(&v_empty[c % kStages]), (c / kStages) & 1))
-          ok = false;
-      }
-      if (!ok) set_status(MD_DEV_TIMEOUT);
+      // Before the CTA may exit, every copy issued into its shared memory has
+      // landed: wait for the last phase of each ring slot's full barriers (TMA
+      // completion, whatever the consumers did) and of the Q barrier. Earlier
+      // copies were consumed before their slot was refilled.
+      bool drained = mbar_wait(smem_u32(q_full), 0);
+      for (int c = (nk > kStages ? nk - kStages : 0); c < nk; ++c)
+        drained = mbar_wait(smem_u32(&k_full[c % kStages]), (c / kStages) & 1) && drained;
+      for (int c = (nv > kStages ? nv - kStages : 0); c < nv; ++c)
+        drained = mbar_wait(smem_u32(&v_full[c % kStages]), (c / kStages) & 1) && drained;
+      if (!ok || !drained) set_status(MD_DEV_TIMEOUT);
     }
   } else if (warp == 1) {
     // ---------------------------------- MMA ----------------------------------
@@ -276,6 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c + kSBufs < nch) ok = issue_s(c + kSBufs);
       }
       if (ok) umma_commit(smem_u32(o_last));
+      // TMEM is released after this CTA's last barrier: every MMA issued so far
+      // (all of them, or those before a wait gave up) must have completed
+      umma_commit(smem_u32(mma_done));
+      if (!mbar_wait(smem_u32(mma_done), 0)) ok = false;
       if (!ok) set_status(MD_DEV_TIMEOUT);
     }
   } else {

@@ -18,8 +18,14 @@ __device__ __forceinline__ void set_status(int bit) { atomicOr(&g_device_status,
 
 // Upper bound on any pipeline wait. A correct launch never comes close (the
 // longest kernel runs for a few milliseconds); after it a kernel flags
-// MD_DEV_TIMEOUT and returns instead of spinning forever.
+// MD_DEV_TIMEOUT and returns instead of spinning forever. md_set_wait_limit
+// changes it (per device).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+// Test hook (md_test_withhold_attention_chunk): chunk index whose K/V copies the
+// tree-attention producers do not issue, or -1.
+__device__ int g_withhold_chunk = -1;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -115,8 +121,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = *const_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit) return false;
   }
   return true;
 }
@@ -217,6 +224,11 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
                : "memory");
   return v;
 }
+__device__ __forceinline__ float ld_cluster_f1(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
@@ -278,6 +290,11 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask
       "h"(cta_mask)
       : "memory");
 }
+
+// Gumbel noise -ln(-ln u) of a uniform u in (0, 1): adding it to logits / tau
+// and keeping the k largest draws k tokens from softmax(logits / tau) without
+// replacement, in draw order (Gumbel-top-k).
+__device__ __forceinline__ float gumbel_noise(float u) { return -logf(-logf(u)); }
 
 // ---------------------------------------------------------------------------
 // Total order used by every top-k / argmax: larger value first, then lower id.

@@ -41,7 +41,8 @@ struct Plan {
   int units;    // K * ntiles
   int nstages;  // phase-2 pipeline depth
   int grid;     // phase-2 CTAs (one candidate list per row, head and CTA)
-  size_t off_zt, off_part, off_cnt, off_cval, off_cid, bytes;
+  int stream_k; // phase 2 split by 64-row stages (balanced) instead of whole units
+  size_t off_zt, off_part, off_cnt, off_tick, off_spart, off_cval, off_cid, bytes;
 };
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -77,6 +78,14 @@ inline Plan make_plan(int M, int d, int V, int K, int kmax, int num_sms) {
   p.off_part = o; o = align256(o + size_t(splits) * K * M * d * 4);
   p.off_cnt = o;  o = align256(o + size_t(K) * p.ntile_o * 4);
   p.grid = std::min(num_sms, p.units);
+  // Whole units over the CTAs leave a tail when they do not divide evenly
+  // (2004 units of a 70B call over 148 CTAs: 13 or 14 each; 501 for one head:
+  // 3 or 4). With at least one unit per CTA, cut the (unit, stage) items
+  // instead: a unit then spans at most two CTAs, whose partial logits the
+  // second to finish adds up.
+  p.stream_k = (p.units > p.grid && p.units % p.grid != 0) ? 1 : 0;
+  p.off_tick = o; o = align256(o + size_t(p.units) * 4);            // one ticket per unit (zeroed with the counters)
+  p.off_spart = o; o = align256(o + size_t(p.grid) * 2 * M * kTileV * 4);
   p.off_cval = o; o = align256(o + size_t(M) * K * p.grid * kmax * 4);
   p.off_cid = o;  o = align256(o + size_t(M) * K * p.grid * kmax * 4);
   p.bytes = o;
@@ -244,10 +253,28 @@ struct VocabArgs {
   float* cand_val;     // [M, K, gridDim.x, kmax]: one list per (row, head, CTA)
   int* cand_id;
   float* logits_dbg;   // [M, K, V] or null
+  const float* gumbel_u;  // [M, K, V] uniforms (sampled drafts) or null (top-k of the logits)
+  float inv_tau;          // 1 / draft temperature (sampled drafts)
+  int stream_k;           // CTA ranges in (unit, stage) items instead of whole units
+  int* tickets;           // [units], zero at launch: a split unit's second finisher adds the parts
+  float* spart;           // [gridDim.x][2][M][256]: partial logits of the units a CTA range cuts
   int d, V, K, kmax, ntiles, units, nstages;
   int shared, kh;      // shared projection: K == 1 and row m is (m / kh, head m % kh)
   int kph[MD_MAX_K];
 };
+
+// This CTA's (unit, stage) items [i0, i1): whole units, or (stream_k) an
+// equal share of the units x stages items.
+__device__ __forceinline__ void item_range(const VocabArgs& a, int S, long long& i0, long long& i1) {
+  if (a.stream_k) {
+    const long long W = (long long)a.units * S;
+    i0 = (long long)blockIdx.x * W / gridDim.x;
+    i1 = (long long)(blockIdx.x + 1) * W / gridDim.x;
+  } else {
+    i0 = (long long)blockIdx.x * a.units / gridDim.x * S;
+    i1 = (long long)(blockIdx.x + 1) * a.units / gridDim.x * S;
+  }
+}
 
 template <int M>
 __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
@@ -283,11 +310,12 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       bool waited_primary = false;
       int it = 0;
       bool ok = true;
-      const int u0 = int((long long)blockIdx.x * a.units / gridDim.x);
-      const int u1 = int((long long)(blockIdx.x + 1) * a.units / gridDim.x);
-      for (int unit = u0; unit < u1 && ok; ++unit) {
+      long long i0, i1;                    // this CTA's (unit, stage) items
+      item_range(a, stages_per_unit, i0, i1);
+      for (long long w = i0; w < i1 && ok; ++w, ++it) {
+        const int unit = int(w / stages_per_unit), s = int(w % stages_per_unit);
         const int k = unit / a.ntiles, tile = unit % a.ntiles;
-        for (int s = 0; s < stages_per_unit; ++s, ++it) {
+        {
           const int slot = it % ns;
           if (it >= ns && !mbar_wait(smem_u32(&empty[slot]), ((it / ns) - 1) & 1)) {
             set_status(MD_DEV_TIMEOUT);
@@ -319,14 +347,19 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
   }
 
   // -------------------------------- consumers --------------------------------
+  __shared__ int s_ticket;
   int it = 0;
   bool ok = true;
-  const int u0 = int((long long)blockIdx.x * a.units / gridDim.x);
-  const int u1 = int((long long)(blockIdx.x + 1) * a.units / gridDim.x);
+  long long i0, i1;
+  item_range(a, stages_per_unit, i0, i1);
   // Running top-k of (row m = warp, current head): lane r holds entry r.
   float rv = -INFINITY;
   int ri = INT_MAX;
-  for (int unit = u0; unit < u1; ++unit) {
+  // One part = the stages of one unit that lie in this CTA's range.
+  for (long long w = i0; w < i1;) {
+    const int unit = int(w / stages_per_unit);
+    const int s_lo = int(w % stages_per_unit);
+    const int s_hi = int(min((long long)stages_per_unit, s_lo + (i1 - w)));
     const int k = unit / a.ntiles, tile = unit % a.ntiles;
     float acc[M][8];
 #pragma unroll
@@ -334,7 +367,7 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[m][c] = 0.f;
 
-    for (int s = 0; s < stages_per_unit; ++s, ++it) {
+    for (int s = s_lo; s < s_hi; ++s, ++it) {
       const int slot = it % ns;
       if (ok && !mbar_wait(smem_u32(&full[slot]), (it / ns) & 1)) {
         set_status(MD_DEV_TIMEOUT);
@@ -345,10 +378,10 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
         const uint8_t* zb = stage_z + size_t(slot) * kStageZBytes + warp * 8 * 16;
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          const uint4 w = *reinterpret_cast<const uint4*>(wb + r * (kTileV * 2));
+          const uint4 wv = *reinterpret_cast<const uint4*>(wb + r * (kTileV * 2));
           const uint4 zv = *reinterpret_cast<const uint4*>(zb + r * 16);
           const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const float zm = (m & 1) ? bf16hi(zw[m >> 1]) : bf16lo(zw[m >> 1]);
@@ -363,6 +396,8 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
     }
+    w += s_hi - s_lo;
+    const bool whole = s_lo == 0 && s_hi == stages_per_unit;
 
     // Cross-warp reduction in fixed warp order.
 #pragma unroll
@@ -372,17 +407,50 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       dst[1] = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
     }
     named_bar_sync(1, kConsumerWarps * 32);
-    {
-      const int t = threadIdx.x;  // 0..255: one column each
+    const int t = threadIdx.x;  // 0..255: one column each
+    float v[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float x = 0.f;
+#pragma unroll
+      for (int wp = 0; wp < kConsumerWarps; ++wp) x += red[(size_t(wp) * M + m) * kTileV + t];
+      v[m] = x;
+    }
+    bool fold = whole;
+    if (!whole) {
+      // A unit cut by the range: the part holding stage 0 sits at the end of
+      // one CTA's range (its slot 1), the rest at the start of the next CTA's
+      // (its slot 0). Each writes its partial logits; the second to finish
+      // adds first part + second part, in that order, and folds the unit.
+      const bool head_part = s_lo == 0;
+      float* mine = a.spart + ((size_t(blockIdx.x) * 2 + (head_part ? 1 : 0)) * M) * kTileV;
+#pragma unroll
+      for (int m = 0; m < M; ++m) mine[m * kTileV + t] = v[m];
+      __threadfence();
+      named_bar_sync(1, kConsumerWarps * 32);
+      if (t == 0) s_ticket = atomicAdd(&a.tickets[unit], 1);
+      named_bar_sync(1, kConsumerWarps * 32);
+      fold = s_ticket == 1;
+      if (fold) {
+        __threadfence();
+        const float* other = a.spart + ((size_t(blockIdx.x + (head_part ? 1 : -1)) * 2 + (head_part ? 0 : 1)) * M) *
+                                           kTileV;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float o = __ldcg(other + m * kTileV + t);
+          v[m] = head_part ? v[m] + o : o + v[m];
+        }
+      }
+    }
+    if (fold) {
       const int col = tile * kTileV + t;
 #pragma unroll
       for (int m = 0; m < M; ++m) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) v += red[(size_t(w) * M + m) * kTileV + t];
         if (col < a.V) {
-          lg[m * kTileV + t] = v;
-          if (a.logits_dbg) a.logits_dbg[(size_t(m) * a.K + k) * a.V + col] = v;
+          const size_t idx = (size_t(m) * a.K + k) * a.V + col;
+          if (a.logits_dbg) a.logits_dbg[idx] = v[m];
+          // sampled drafts rank the Gumbel keys logit / tau - ln(-ln u) instead
+          lg[m * kTileV + t] = a.gumbel_u ? fmaf(v[m], a.inv_tau, gumbel_noise(__ldg(a.gumbel_u + idx))) : v[m];
         } else {
           lg[m * kTileV + t] = -INFINITY;
         }
@@ -395,53 +463,56 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
     // order among the tile's 256 logits and the running list.
     if (warp < M) {
       const int m = warp;
-      float v[kTileV / 32];
-      int id[kTileV / 32];
-#pragma unroll
-      for (int i = 0; i < kTileV / 32; ++i) {
-        const int c = lane + 32 * i;
-        v[i] = lg[m * kTileV + c];
-        id[i] = (tile * kTileV + c < a.V) ? tile * kTileV + c : INT_MAX;
-      }
-      float pv = INFINITY;
-      int pid = -1;
       const int kk = param_at(a.kph, a.shared ? m % a.kh : k);
-      float nrv = -INFINITY;
-      int nri = INT_MAX;
-      for (int r = 0; r < kk; ++r) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
+      if (fold) {
+        float vv[kTileV / 32];
+        int id[kTileV / 32];
 #pragma unroll
         for (int i = 0; i < kTileV / 32; ++i) {
-          if (better(pv, pid, v[i], id[i]) && better(v[i], id[i], bv, bi)) {
-            bv = v[i];
-            bi = id[i];
-          }
+          const int c = lane + 32 * i;
+          vv[i] = lg[m * kTileV + c];
+          id[i] = (tile * kTileV + c < a.V) ? tile * kTileV + c : INT_MAX;
         }
-        if (better(pv, pid, rv, ri) && better(rv, ri, bv, bi)) {
-          bv = rv;
-          bi = ri;
-        }
+        float pv = INFINITY;
+        int pid = -1;
+        float nrv = -INFINITY;
+        int nri = INT_MAX;
+        for (int r = 0; r < kk; ++r) {
+          float bv = -INFINITY;
+          int bi = INT_MAX;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (better(ov, oi, bv, bi)) {
-            bv = ov;
-            bi = oi;
+          for (int i = 0; i < kTileV / 32; ++i) {
+            if (better(pv, pid, vv[i], id[i]) && better(vv[i], id[i], bv, bi)) {
+              bv = vv[i];
+              bi = id[i];
+            }
           }
+          if (better(pv, pid, rv, ri) && better(rv, ri, bv, bi)) {
+            bv = rv;
+            bi = ri;
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (better(ov, oi, bv, bi)) {
+              bv = ov;
+              bi = oi;
+            }
+          }
+          if (lane == r) {
+            nrv = bv;
+            nri = bi;
+          }
+          pv = bv;
+          pid = bi;
         }
-        if (lane == r) {
-          nrv = bv;
-          nri = bi;
-        }
-        pv = bv;
-        pid = bi;
+        rv = nrv;
+        ri = nri;
       }
-      rv = nrv;
-      ri = nri;
-      // flush the list when the next unit belongs to another head (or there is none)
-      if (unit + 1 == u1 || (unit + 1) / a.ntiles != k) {
+      // flush the list when the range moves to another head (or ends): every
+      // CTA whose range meets head k writes a list for it, empty or not
+      if (w >= i1 || int(w / stages_per_unit) / a.ntiles != k) {
         if (lane < kk) {
           const size_t cb = ((size_t(m) * a.K + k) * gridDim.x + blockIdx.x) * a.kmax + lane;
           a.cand_val[cb] = rv;
@@ -475,6 +546,7 @@ struct MergeArgs {
   float* topk_vals;
   int K, kmax, nslots;
   int partitioned, units, ntiles;   // producer partition (partitioned == 1)
+  int stages;          // > 0: the producer cut units x stages items (stages per unit), not whole units
   int kh;              // heads for the top-k size: row mk uses kph[mk % kh]
   int kph[MD_MAX_K];
 };
@@ -503,8 +575,11 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
     const int c = c0 + threadIdx.x;
     bool rel = c < a.nslots;
     if (rel && a.partitioned) {
-      const long long u0 = (long long)c * a.units / a.nslots, u1 = (long long)(c + 1) * a.units / a.nslots;
-      rel = u1 > (long long)k * a.ntiles && u0 < (long long)(k + 1) * a.ntiles;
+      const long long S = a.stages > 0 ? a.stages : 1;     // items per unit
+      const long long W = (long long)a.units * S;
+      const long long w0 = a.stages > 0 ? (long long)c * W / a.nslots : (long long)c * a.units / a.nslots;
+      const long long w1 = a.stages > 0 ? (long long)(c + 1) * W / a.nslots : (long long)(c + 1) * a.units / a.nslots;
+      rel = w1 > (long long)k * a.ntiles * S && w0 < (long long)(k + 1) * a.ntiles * S;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, rel);
     if (lane == 0) warp_cnt[warp] = __popc(bal);

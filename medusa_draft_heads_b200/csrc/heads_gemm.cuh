@@ -61,6 +61,8 @@ struct Args {
   float* cand_val;                // [M, K, per_mt, kmax]  phase 2: one list per (row, head, CTA of the row tile)
   int* cand_id;
   float* logits_dbg;              // [M, K, N] or null
+  const float* gumbel_u;          // phase 2: [M, K, N] uniforms (sampled drafts) or null
+  float inv_tau;                  // phase 2: 1 / draft temperature (sampled drafts)
   int kmax;
   int zg_mk;                      // phase 1: write z rows in (row, head) order [M*K, d]
   int kh;                         // phase 2: row m uses kph[m % kh] when K == 1 (shared projection)
@@ -122,17 +124,32 @@ __device__ __forceinline__ void silu_residual_store(const Args& a, int m, int k,
 
 // Phase-2 epilogue for 32 logits of row m, head k, columns c0..: fold them
 // into the running top-k (and copy them out when the debug logits are kept).
+// Sampled drafts fold the Gumbel keys logit / tau - ln(-ln u) instead.
 __device__ __forceinline__ void topk_tile_columns(const Args& a, SmemList& L, int m, int k, int c0,
                                                   const float (&v)[32]) {
-#pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (c0 + j < a.N && better(v[j], c0 + j, L.tv, L.ti)) L.insert(v[j], c0 + j);
+  const size_t base = (size_t(m) * a.K + k) * a.N + c0;
   if (a.logits_dbg) {
-    float* lp = a.logits_dbg + (size_t(m) * a.K + k) * a.N + c0;
+    float* lp = a.logits_dbg + base;
 #pragma unroll
     for (int j = 0; j < 32; j += 4)
       if (c0 + j < a.N) *reinterpret_cast<float4*>(lp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
   }
+  if (a.gumbel_u) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      if (c0 + j >= a.N) break;
+      const float4 u = __ldg(reinterpret_cast<const float4*>(a.gumbel_u + base + j));
+      const float key[4] = {fmaf(v[j], a.inv_tau, gumbel_noise(u.x)), fmaf(v[j + 1], a.inv_tau, gumbel_noise(u.y)),
+                            fmaf(v[j + 2], a.inv_tau, gumbel_noise(u.z)), fmaf(v[j + 3], a.inv_tau, gumbel_noise(u.w))};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (better(key[e], c0 + j + e, L.tv, L.ti)) L.insert(key[e], c0 + j + e);
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (c0 + j < a.N && better(v[j], c0 + j, L.tv, L.ti)) L.insert(v[j], c0 + j);
 }
 
 // Write a running list to candidate slot `slot` of (row m, head k).

@@ -19,6 +19,7 @@
 #include "accept.cuh"
 #include "commit.cuh"
 #include "hydra.cuh"
+#include "reject.cuh"
 
 struct md_tree {
   md::TreeParams tp;
@@ -123,7 +124,7 @@ md_status set_smem(Kernel k, int bytes) {
 template <int M>
 md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
                        const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
-                       uint8_t* ws, cudaStream_t st) {
+                       const float* gumbel_u, float inv_tau, uint8_t* ws, cudaStream_t st) {
   using namespace md::heads;
   md_status s;
   // phase 1
@@ -134,7 +135,8 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   wa.counters = reinterpret_cast<int*>(ws + pl.off_cnt);
   wa.d = pl.d; wa.K = pl.K; wa.splits = pl.splits; wa.rows = pl.rows; wa.ntile_o = pl.ntile_o;
   wa.shared = 0;
-  if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, size_t(pl.K) * pl.ntile_o * 4, st))) != MD_OK) return s;
+  // phase-1 counters and phase-2 tickets are contiguous: one memset
+  if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, pl.off_spart - pl.off_cnt, st))) != MD_OK) return s;
   const int w1_smem = pl.rows * 16 + kConsumerWarps * M * kW1TileO * 4;
   if ((s = set_smem(heads_w1_kernel<M>, w1_smem)) != MD_OK) return s;
   heads_w1_kernel<M><<<dim3(pl.ntile_o, pl.splits, pl.K), kW1Threads, w1_smem, st>>>(wa);
@@ -148,6 +150,11 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   va.cand_val = reinterpret_cast<float*>(ws + pl.off_cval);
   va.cand_id = reinterpret_cast<int*>(ws + pl.off_cid);
   va.logits_dbg = logits_dbg;
+  va.gumbel_u = gumbel_u;
+  va.inv_tau = inv_tau;
+  va.stream_k = pl.stream_k;
+  va.tickets = reinterpret_cast<int*>(ws + pl.off_tick);
+  va.spart = reinterpret_cast<float*>(ws + pl.off_spart);
   va.d = pl.d; va.V = pl.V; va.K = pl.K; va.kmax = pl.kmax; va.ntiles = pl.ntiles; va.units = pl.units;
   va.nstages = pl.nstages;
   va.shared = 0; va.kh = pl.K;
@@ -172,6 +179,7 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = pl.K; ma.kmax = pl.kmax; ma.nslots = pl.grid;
   ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.kh = pl.K;
+  ma.stages = va.stream_k ? pl.d / kStageRows : 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
   return launch_pdl(heads_merge_kernel, dim3(pl.M * pl.K), dim3(256), 0, st, ma);
 }
@@ -301,7 +309,8 @@ md_status launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const md
 template <int KK>
 md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16* h, const md_bf16* W1,
                             const md_bf16* b1, const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids,
-                            float* topk_vals, float* logits_dbg, uint8_t* ws, cudaStream_t st) {
+                            float* topk_vals, float* logits_dbg, const float* gumbel_u, float inv_tau, uint8_t* ws,
+                            cudaStream_t st) {
   using namespace md::gemm;
   const GemmPlan pl = gemm_plan(M, d, V, K, kmax);
   md_status s;
@@ -325,6 +334,8 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   if ((s = make_map_3d_sw128(&amap, ga.zg, d, M, K, kBK, kBM)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&bmap, Wv, V, d, K, 64, kBK)) != MD_OK) return s;
   ga.N = V; ga.ntiles = pl.ntiles2; ga.per_mt = pl.per_mt2; ga.groups = pl.groups; ga.a_shared = 0;
+  ga.gumbel_u = gumbel_u;
+  ga.inv_tau = inv_tau;
   if ((s = launch_gemm<EPI_TOPK, KK>(amap, bmap, ga, pl.grid2, pl.cluster, true, st)) != MD_OK) return s;
 
   // phase 3: merge the tiles' candidates
@@ -333,6 +344,7 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = K; ma.kmax = kmax; ma.nslots = pl.per_mt2;
   ma.partitioned = 1; ma.units = K * pl.ntiles2; ma.ntiles = pl.ntiles2; ma.kh = K;
+  ma.stages = 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
   return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
 }
@@ -346,6 +358,7 @@ struct SharedPlan {
   md::heads::Plan p1, p2;      // streaming: phase-1 plan (M rows, K heads), phase-2 plan (M*K rows, 1 head)
   GemmPlan g1, g2;             // tensor cores: phase 1 (M rows, K heads), phase 2 (M*K rows, 1 head)
   size_t off2, bytes;
+  size_t tick2, spart2, cval2, cid2;   // streaming: phase-2 tickets, partials, candidates (from off2)
 };
 
 SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
@@ -355,8 +368,12 @@ SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
   if (p.stream) {
     p.p1 = md::heads::make_plan(M, d, V, K, kmax, num_sms());
     p.p2 = md::heads::make_plan(M * K, d, V, 1, kmax, num_sms());
-    p.off2 = align256(p.p1.off_cval);                    // phase-2 candidates after phase-1 data
-    p.bytes = p.off2 + (p.p2.bytes - p.p2.off_cval);
+    p.off2 = align256(p.p1.off_cval);                    // phase-2 data after phase-1 data
+    p.tick2 = 0;
+    p.spart2 = p.p2.off_spart - p.p2.off_tick;
+    p.cval2 = p.p2.off_cval - p.p2.off_tick;
+    p.cid2 = p.p2.off_cid - p.p2.off_tick;
+    p.bytes = p.off2 + (p.p2.bytes - p.p2.off_tick);
   } else {
     p.g1 = gemm_plan(M, d, V, K, kmax);                   // z [M*K, d] lives at g1.off_z
     p.g2 = gemm_plan(M * K, d, V, 1, kmax);
@@ -382,6 +399,8 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   wa.d = p1.d; wa.K = p1.K; wa.splits = p1.splits; wa.rows = p1.rows; wa.ntile_o = p1.ntile_o;
   wa.shared = 1;
   if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, size_t(p1.K) * p1.ntile_o * 4, st))) != MD_OK) return s;
+  // phase-2 tickets of the shared projection (its own plan p2)
+  if ((s = cuda_ok(cudaMemsetAsync(ws + sp.off2 + sp.tick2, 0, size_t(p2.units) * 4, st))) != MD_OK) return s;
   auto run_w1 = [&](auto kern, int smem) -> md_status {
     md_status r;
     if ((r = set_smem(kern, smem)) != MD_OK) return r;
@@ -400,9 +419,14 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   if ((s = make_map_2d(&map, Wv, uint64_t(p2.V), uint64_t(p2.d), kTileV, kStageRows)) != MD_OK) return s;
   VocabArgs va;
   va.zt = wa.zt;
-  va.cand_val = reinterpret_cast<float*>(ws + sp.off2);
-  va.cand_id = reinterpret_cast<int*>(ws + sp.off2 + (p2.off_cid - p2.off_cval));
+  va.cand_val = reinterpret_cast<float*>(ws + sp.off2 + sp.cval2);
+  va.cand_id = reinterpret_cast<int*>(ws + sp.off2 + sp.cid2);
   va.logits_dbg = logits_dbg;
+  va.gumbel_u = nullptr;
+  va.inv_tau = 1.f;
+  va.stream_k = p2.stream_k;
+  va.tickets = reinterpret_cast<int*>(ws + sp.off2 + sp.tick2);
+  va.spart = reinterpret_cast<float*>(ws + sp.off2 + sp.spart2);
   va.d = p2.d; va.V = p2.V; va.K = 1; va.kmax = p2.kmax; va.ntiles = p2.ntiles; va.units = p2.units;
   va.nstages = p2.nstages;
   va.shared = 1; va.kh = p1.K;
@@ -417,6 +441,7 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = 1; ma.kmax = p2.kmax; ma.nslots = p2.grid;
   ma.partitioned = 1; ma.units = p2.units; ma.ntiles = p2.ntiles; ma.kh = p1.K;
+  ma.stages = va.stream_k ? p2.d / kStageRows : 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
   return launch_pdl(heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
 }
@@ -454,6 +479,7 @@ md_status launch_heads_shared_gemm(const SharedPlan& sp, int M, int d, int V, in
   ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
   ma.K = 1; ma.kmax = kmax; ma.nslots = sp.g2.per_mt2;
   ma.partitioned = 1; ma.units = sp.g2.ntiles2; ma.ntiles = sp.g2.ntiles2; ma.kh = K;
+  ma.stages = 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
   return launch_pdl(md::heads::heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
 }
@@ -648,6 +674,49 @@ md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPl
   return MD_OK;
 }
 
+// md_medusa_heads and md_medusa_heads_sampled: checks, then the streaming
+// (M <= 4) or tensor-core path. gumbel_u null: top-k of the logits; else the
+// top-k of the Gumbel keys logit * inv_tau - ln(-ln u).
+md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, int32_t M,
+                     int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax, int32_t* topk_ids,
+                     float* topk_vals, float* logits_dbg, const float* gumbel_u, float inv_tau, void* ws,
+                     size_t ws_bytes, void* stream) {
+  if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
+  md_status s = heads_check(M, d, V, K, kmax);
+  if (s != MD_OK) return s;
+  for (int k = 0; k < K; ++k)
+    if (k_per_head[k] < 1 || k_per_head[k] > kmax || k_per_head[k] > V) return MD_ERR_INVALID_ARG;
+  if (!aligned(h, 2) || !aligned(W1, 16) || !aligned(b1, 2) || !aligned(Wv, 16) || !aligned(topk_ids, 4) ||
+      !aligned(topk_vals, 4) || (logits_dbg && !aligned(logits_dbg, 4)))
+    return MD_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  if (M > md::heads::kMaxM) {
+    // tensor-core path: h, W1, Wv feed TMA directly (16-byte aligned rows: d % 64, V % 8)
+    if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < gemm_plan(M, d, V, K, kmax).bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+    int mk = 0;
+    for (int k = 0; k < K; ++k) mk = std::max(mk, int(k_per_head[k]));
+    if (mk <= 4)
+      return launch_heads_gemm<4>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg,
+                                  gumbel_u, inv_tau, w, st);
+    if (mk <= 8)
+      return launch_heads_gemm<8>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg,
+                                  gumbel_u, inv_tau, w, st);
+    return launch_heads_gemm<16>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg,
+                                 gumbel_u, inv_tau, w, st);
+  }
+  const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
+  if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+  switch (M) {
+    case 1: return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
+    case 2: return launch_heads<2>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
+    case 3: return launch_heads<3>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
+    case 4: return launch_heads<4>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
+    default: return MD_ERR_UNSUPPORTED;
+  }
+}
+
 // Scratch of md_medusa_heads_static: a fixed array in the library's device
 // image (every GPU that loads the library holds it until the process exits).
 __device__ __align__(256) uint8_t g_heads_static_scratch[MD_HEADS_STATIC_SCRATCH_BYTES];
@@ -746,37 +815,19 @@ md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1
                           int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax,
                           int32_t* topk_ids, float* topk_vals, float* logits_dbg, void* ws, size_t ws_bytes,
                           void* stream) {
-  if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
-  md_status s = heads_check(M, d, V, K, kmax);
-  if (s != MD_OK) return s;
-  for (int k = 0; k < K; ++k)
-    if (k_per_head[k] < 1 || k_per_head[k] > kmax || k_per_head[k] > V) return MD_ERR_INVALID_ARG;
-  if (!aligned(h, 2) || !aligned(W1, 16) || !aligned(b1, 2) || !aligned(Wv, 16) || !aligned(topk_ids, 4) ||
-      !aligned(topk_vals, 4) || (logits_dbg && !aligned(logits_dbg, 4)))
-    return MD_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  if (M > md::heads::kMaxM) {
-    // tensor-core path: h, W1, Wv feed TMA directly (16-byte aligned rows: d % 64, V % 8)
-    if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
-    if (!ws || ws_bytes < gemm_plan(M, d, V, K, kmax).bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
-    int mk = 0;
-    for (int k = 0; k < K; ++k) mk = std::max(mk, int(k_per_head[k]));
-    if (mk <= 4)
-      return launch_heads_gemm<4>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    if (mk <= 8)
-      return launch_heads_gemm<8>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    return launch_heads_gemm<16>(M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-  }
-  const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
-  if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
-  switch (M) {
-    case 1: return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 2: return launch_heads<2>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 3: return launch_heads<3>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    case 4: return launch_heads<4>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-    default: return MD_ERR_UNSUPPORTED;
-  }
+  return heads_call(h, W1, b1, Wv, M, d, V, K, k_per_head, kmax, topk_ids, topk_vals, logits_dbg, nullptr, 1.f, ws,
+                    ws_bytes, stream);
+}
+
+md_status md_medusa_heads_sampled(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
+                                  int32_t M, int32_t d, int32_t V, int32_t K, const int32_t* k_per_head,
+                                  int32_t kmax, float temperature, const float* uniforms, int32_t* topk_ids,
+                                  float* topk_keys, float* logits, void* ws, size_t ws_bytes, void* stream) {
+  if (!uniforms || !logits) return MD_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !std::isfinite(temperature)) return MD_ERR_INVALID_ARG;
+  if (!aligned(uniforms, 16) || !aligned(logits, 16)) return MD_ERR_INVALID_ARG;
+  return heads_call(h, W1, b1, Wv, M, d, V, K, k_per_head, kmax, topk_ids, topk_keys, logits, uniforms,
+                    1.0f / temperature, ws, ws_bytes, stream);
 }
 
 md_status md_heads_shared_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax, size_t* bytes) {
@@ -827,9 +878,13 @@ md_status md_medusa_heads_shared(const md_bf16* h, const md_bf16* W1, const md_b
 md_status md_medusa_heads_static(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
                                  int32_t M, int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax,
                                  int32_t* topk_ids, float* topk_vals, float* logits_dbg, void* stream) {
+  // the argument checks of md_medusa_heads come before the scratch-size check
+  if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
   size_t need = 0;
   md_status s = md_heads_workspace(M, d, V, K, kmax, &need);
   if (s != MD_OK) return s;
+  for (int k = 0; k < K; ++k)
+    if (k_per_head[k] < 1 || k_per_head[k] > kmax || k_per_head[k] > V) return MD_ERR_INVALID_ARG;
   if (need > size_t(MD_HEADS_STATIC_SCRATCH_BYTES)) return MD_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((s = static_scratch_address(&scratch)) != MD_OK) return s;
@@ -1045,6 +1100,55 @@ md_status md_tree_accept_sampled(const float* logits, int32_t V, const int32_t* 
   return launch_pdl(md::acc::accept_walk_kernel, dim3(B), dim3(MD_MAX_T), 0, st, tree->tp, a);
 }
 
+md_status md_tree_accept_rejection(const float* logits, int32_t V, const int32_t* tokens, const md_tree* tree,
+                                   int32_t B, int32_t K, float temperature, const float* head_logits, int32_t M,
+                                   int32_t Kh, const int32_t* head_row, float temperature_q, const float* u_accept,
+                                   const float* u_residual, int32_t* accept_len, int32_t* path, int32_t* bonus,
+                                   void* stream) {
+  using namespace md::rej;
+  if (!logits || !tokens || !tree || !head_logits || !u_accept || !u_residual || !accept_len || !path || !bonus)
+    return MD_ERR_INVALID_ARG;
+  const TreeParams& tp = tree->tp;
+  if (B < 1 || V < 1 || M < 1 || K < tp.max_depth || K > MD_MAX_K || Kh < tp.max_depth) return MD_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !std::isfinite(temperature) || !(temperature_q > 0.f) || !std::isfinite(temperature_q))
+    return MD_ERR_INVALID_ARG;
+  const int slice = (V + kCtas - 1) / kCtas;
+  if (slice > kMaxSlice) return MD_ERR_UNSUPPORTED;
+  // the children of every node must carry the ranks 0 .. m-1 (the first m draws)
+  for (int t = 0; t < tp.T; ++t) {
+    int m = 0, rmax = -1;
+    for (int j = 1; j < tp.T; ++j)
+      if (tp.parent[j] == t) {
+        ++m;
+        rmax = std::max(rmax, int(tp.rank[j]));
+      }
+    if (m > 0 && rmax != m - 1) return MD_ERR_UNSUPPORTED;
+  }
+  Args a;
+  a.logits = logits; a.head_logits = head_logits; a.head_row = head_row; a.tokens = tokens;
+  a.u_acc = u_accept; a.u_res = u_residual; a.accept_len = accept_len; a.path = path; a.bonus = bonus;
+  a.V = V; a.T = tp.T; a.K = K; a.M = M; a.Kh = Kh; a.slice = slice;
+  a.inv_tau = 1.0f / temperature;
+  a.inv_tau_q = 1.0f / temperature_q;
+  md_status s;
+  if ((s = set_smem(reject_accept_kernel, kSmem)) != MD_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kCtas, B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, reject_accept_kernel, tp, a));
+}
+
 md_status md_tree_commit(md_bf16* k_cache, md_bf16* v_cache, int32_t S_max, int32_t Hkv, int32_t dh,
                          const md_tree* tree, int32_t B, const int32_t* prefix_len, const int32_t* accept_len,
                          const int32_t* path, int32_t K, const int32_t* bonus, int32_t* new_prefix_len,
@@ -1077,6 +1181,17 @@ md_status md_get_device_status(void* stream, int32_t* out, int32_t clear) {
     if ((s = cuda_ok(cudaMemcpyToSymbol(md::g_device_status, &zero, sizeof(int)))) != MD_OK) return s;
   }
   return MD_OK;
+}
+
+md_status md_set_wait_limit(uint64_t ns) {
+  const unsigned long long v = ns == 0 ? md::kWaitLimitNs : (unsigned long long)ns;
+  return cuda_ok(cudaMemcpyToSymbol(md::g_wait_limit_ns, &v, sizeof(v)));
+}
+
+md_status md_test_withhold_attention_chunk(int32_t chunk) {
+  if (chunk < -1) return MD_ERR_INVALID_ARG;
+  const int v = chunk;
+  return cuda_ok(cudaMemcpyToSymbol(md::g_withhold_chunk, &v, sizeof(v)));
 }
 
 const char* md_status_string(md_status status) {

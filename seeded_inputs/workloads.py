@@ -33,7 +33,7 @@ class Workload:
     w_sigma: float = 0.02       # head weights ~ N(0, 0.02)
     logit_sigma: float = 1.0    # target logits ~ N(0, logit_sigma)
     bump: float = 1.0           # planted argmax margin over the row maximum
-    mode: str = "greedy"        # or "typical", "sample"
+    mode: str = "greedy"        # or "typical", "sample", "rejection"
     temperature: float = 0.7
     eps: float = 0.09
     alpha: float = 0.3
@@ -86,8 +86,12 @@ LLAMA70B_SHARED = replace(LLAMA70B, name="llama3-70b-shared-proj", shared_vocab=
 # The same 70B step with lossless sampled acceptance (temperature 0.7).
 LLAMA70B_SAMPLED = replace(LLAMA70B, name="llama3-70b-sampled", mode="sample", temperature=0.7)
 
+# The same 70B step with candidates drawn from the heads' own distributions and
+# lossless acceptance by rejection sampling (temperature 0.7 for both).
+LLAMA70B_REJECTION = replace(LLAMA70B, name="llama3-70b-rejection", mode="rejection", temperature=0.7)
+
 WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS, PROF_GEMM,
-                                 LLAMA70B_SHARED, LLAMA70B_SAMPLED)}
+                                 LLAMA70B_SHARED, LLAMA70B_SAMPLED, LLAMA70B_REJECTION)}
 
 
 def sweep_8b(B: int, tree: str, prefix: int, mode: str = "greedy") -> Workload:

@@ -100,6 +100,23 @@ def test_workspace_queries_and_unsupported_sizes(libmedusa):
     assert libmedusa.md_accept_workspace(1, 129, 128256, ctypes.byref(n)) == -2
 
 
+def test_static_heads_checks_arguments_before_scratch_size(libmedusa):
+    """md_medusa_heads_static rejects null pointers and bad per-head k as
+    md_medusa_heads does, even for a shape whose scratch would not fit; only
+    valid arguments reach the size check. Nothing is launched on either path."""
+    fn = libmedusa.md_medusa_heads_static
+    P, I = ctypes.c_void_p, ctypes.c_int32
+    fn.argtypes = [P, P, P, P, I, I, I, I, P, I, P, P, P, P]
+    fn.restype = I
+    kph = _i32([10, 10, 10, 10])
+    fake = ctypes.c_void_p(4096)          # never dereferenced: the call returns before any launch
+    big = (128, 8192, 128256, 4)          # scratch far beyond the 8 MiB array
+    assert fn(None, fake, fake, fake, *big, kph, 10, fake, fake, None, None) == -1
+    assert fn(fake, fake, fake, fake, *big, None, 10, fake, fake, None, None) == -1
+    assert fn(fake, fake, fake, fake, *big, _i32([10, 10, 11, 10]), 10, fake, fake, None, None) == -1
+    assert fn(fake, fake, fake, fake, *big, kph, 10, fake, fake, None, None) == -4
+
+
 @pytest.mark.parametrize("kph,a,n", [((4, 3, 2, 2), TREE_ACCEPT, 16), ((10, 10, 10, 10), TREE_ACCEPT, 64),
                                      ((10, 10, 10, 10), TREE_ACCEPT, 16), ((1, 1, 1, 1), CHAIN_ACCEPT, 4),
                                      ((5, 4, 3), (0.9, 0.5, 0.5), 40), ((3, 3, 3, 3), (1.0, 1.0, 0.5, 0.5), 30)])

@@ -95,6 +95,8 @@ def _attention_case(seed, tups, B, Hq, Hkv, dh, P, S_max, scale=0.0):
     ("g12-cuda-core", ((10, 10, 10, 10), 64), 1, 12, 1, 64, [1000]),
     # long prefix: many key chunks per split, B = 4 with ragged lengths
     ("long-ragged", ((10, 10, 10, 10), 64), 4, 32, 8, 128, [1024, 8191, 333, 5000]),
+    # 9 row tiles per KV head (more than a portable cluster): one CTA per tile, no multicast
+    ("g16-9tiles", ((10, 10, 10, 10), 64), 2, 16, 1, 64, [700, 2100]),
 ])
 def test_tree_attention_matches_oracle(name, tree, B, Hq, Hkv, dh, P):
     kph, n = tree
@@ -124,10 +126,10 @@ def test_tree_attention_70b_sampled_rows():
 
 @pytest.mark.parametrize("S_max", [128, 1024])
 def test_tree_attention_bad_prefix_sets_status_and_zeros(S_max):
-    """A prefix that leaves no room for the tree zeroes that request only. With
-    S_max = 1024 the key range is cut into 8 splits (one cluster per tile):
-    the bad request's splits all hold nothing, and the good request's keys
-    fall in its first split only."""
+    """A prefix that leaves no room for the tree zeroes that request only: it
+    owns no work units, and the merge kernel writes its rows as zeros. With
+    S_max = 1024 the valid first case spreads each tile's chunks over several
+    CTAs, whose partials the merge kernel combines."""
     tups = ot.select_tree((4, 3, 2, 2), TREE_ACCEPT, 16)
     md.device_status(clear=True)
     out, _ = _attention_case(3, tups, 2, 4, 2, 64, np.array([S_max - 28, 60]), S_max)   # P + 17 <= S_max: valid
