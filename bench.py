@@ -222,6 +222,20 @@ class ClockSampler:
 # --------------------------------------------------------------------------- #
 # The oracle on a bounded sample (cpu_baseline leg and --impl reference).
 # --------------------------------------------------------------------------- #
+def _weight_columns(key, k, n_in, n_out, cols, sigma):
+    """Rows 0 .. n_in-1 of head k's [n_in, n_out] weight at the columns `cols`
+    (bf16 bits), drawn from the counter-based generator in row blocks so the
+    index arrays stay small."""
+    cols = np.asarray(cols, dtype=np.uint64)[None, :]
+    out = np.empty((n_in, cols.shape[1]), dtype=np.uint16)
+    step = max(1, (1 << 23) // cols.shape[1])
+    for i0 in range(0, n_in, step):
+        ii = np.arange(i0, min(n_in, i0 + step), dtype=np.uint64)[:, None]
+        idx = (np.uint64(k) * np.uint64(n_in) + ii) * np.uint64(n_out) + cols
+        out[i0:i0 + ii.shape[0]] = gen.normal_bf16_at(key, idx.ravel(), sigma).reshape(ii.shape[0], -1)
+    return out
+
+
 class OracleSampler:
     """Times the CPU oracle on a fraction `frac` of the step's column/row work
     and scales it back to one whole step. Inputs are drawn on the host from
@@ -236,13 +250,10 @@ class OracleSampler:
         rng = np.random.default_rng(1234)
         self.cols_o = np.sort(rng.choice(d, max(1, int(round(d * frac))), replace=False))
         self.cols_v = np.sort(rng.choice(V, max(1, int(round(V * frac))), replace=False))
-        kw = [gen.stream_key(s, n) for n in ("W1", "Wv", "b1", "h")]
-        ii = np.arange(d, dtype=np.uint64)
+        kw = [gen.stream_key(s, n) for n in ("W1", "Wv")]
         # W1[k, i, o] and Wv[k, i, v] at the sampled columns only (counter-based draws)
-        self.W1 = np.stack([gen.normal_bf16_at(kw[0], ((k * d + ii[:, None]) * d + self.cols_o[None, :]).astype(
-            np.uint64).ravel(), w.w_sigma).reshape(d, -1) for k in range(K)])
-        self.Wv = np.stack([gen.normal_bf16_at(kw[1], ((k * d + ii[:, None]) * V + self.cols_v[None, :]).astype(
-            np.uint64).ravel(), w.w_sigma).reshape(d, -1) for k in range(K)])
+        self.W1 = np.stack([_weight_columns(kw[0], k, d, d, self.cols_o, w.w_sigma) for k in range(K)])
+        self.Wv = np.stack([_weight_columns(kw[1], k, d, V, self.cols_v, w.w_sigma) for k in range(K)])
         self.b1 = gen.normal_bf16(s, "b1", (K, d), w.w_sigma)
         self.h = gen.normal_bf16(s, "h", (w.M, d), 1.0)
         self.root = synth.root_tokens(s, w.B, V)
@@ -261,19 +272,29 @@ class OracleSampler:
         tokens = synth.synthetic_tree_tokens(s, w.B, self.parent, V, root_tokens=self.root)
         self.tokens = tokens
         self.logits = synth.planted_logits(s, self.parent, tokens, V, w.accept, sigma=w.logit_sigma, bump=w.bump)
+        # uniforms of the sampled rules; the heads' logits the rejection rule
+        # reads over the whole vocabulary (their values do not change the work)
+        self.u = rng.random((3, w.B, w.T))
+        if w.mode == "rejection":
+            self.u_draft = rng.random((w.M, K, len(self.cols_v)))
+            self.head_logits = rng.normal(0.0, w.logit_sigma, (w.M, K, V))
 
     def step(self):
         """Returns the estimated seconds of one whole oracle step."""
         from oracle import accept as oacc
         from oracle import attention as oa
         from oracle import heads as oh
+        from oracle import rejection as orj
         from oracle import tree as ot
         w = self.w
         t0 = time.perf_counter()
         oh.residual_block_columns(self.h, self.W1, self.b1[:, self.cols_o], self.cols_o)
         t1 = time.perf_counter()
         logits = oh.vocab_logits(self.z, self.Wv)          # self.Wv holds the sampled columns only
-        oh.heads_topk(logits, w.k_per_head, w.kmax)
+        if w.mode == "rejection":
+            orj.sampled_drafts(logits, w.k_per_head, w.kmax, w.temperature, self.u_draft)
+        else:
+            oh.heads_topk(logits, w.k_per_head, w.kmax)
         t2 = time.perf_counter()
         ot.tree_build(self.parent, self.rank, self.topk_ids, self.root, self.P)
         t3 = time.perf_counter()
@@ -281,8 +302,13 @@ class OracleSampler:
         t4 = time.perf_counter()
         if w.mode == "greedy":
             oacc.greedy_accept(self.logits, self.tokens, self.parent, w.K)
-        else:
+        elif w.mode == "typical":
             oacc.typical_accept(self.logits, self.tokens, self.parent, w.K, w.temperature, w.eps, w.alpha)
+        elif w.mode == "sample":
+            oacc.sampled_accept(self.logits, self.tokens, self.parent, w.K, w.temperature, self.u[0])
+        else:
+            orj.rejection_accept(self.logits, self.tokens, self.parent, self.rank, w.K, w.temperature,
+                                 self.head_logits, np.arange(w.B), w.temperature, self.u[1], self.u[2])
         t5 = time.perf_counter()
         return (t1 - t0) / self.frac + (t2 - t1) / self.frac + (t3 - t2) + (t4 - t3) / self.frac + (t5 - t4)
 
@@ -320,6 +346,25 @@ def run_reference(args, w):
                              "host_cpus": os.cpu_count(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_oracle_check(args, w):
+    """One whole (unsampled) oracle step of the workload beside the sampled
+    estimate that the cpu_baseline and reference legs report, so the 1/frac
+    scaling of the sampled step can be checked against the real thing."""
+    t0 = time.perf_counter()
+    full = OracleSampler(w, 1.0)
+    setup = time.perf_counter() - t0
+    full_s = [full.step() for _ in range(args.oracle_check_steps)]
+    del full
+    smp = OracleSampler(w, args.cpu_frac)
+    smp.step()
+    est = [smp.step() for _ in range(5)]
+    unsampled, sampled = float(np.median(full_s)), float(np.median(est))
+    print(json.dumps({"oracle_check": w.name, "unsampled_step_s": unsampled, "unsampled_steps": full_s,
+                      "sampled_estimate_s": sampled, "frac": args.cpu_frac, "estimate_over_unsampled":
+                      sampled / unsampled, "setup_s": setup, "cores": blas_threads(),
+                      "host_cpus": os.cpu_count()}), flush=True)
 
 
 def config_dict(w, P):
@@ -847,12 +892,18 @@ def main():
     ap.add_argument("--cpu-frac", type=float, default=1 / 64)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-frac", type=float, default=1 / 512)
+    ap.add_argument("--oracle-check", action="store_true",
+                    help="time whole (unsampled) oracle steps beside the sampled estimate, then exit (CPU only)")
+    ap.add_argument("--oracle-check-steps", type=int, default=2)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per heads call from an ncu capture of the current kernels")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.oracle_check:
+        run_oracle_check(args, w)
+        return
     if args.sweep:
         run_sweep(args)
         return

@@ -58,6 +58,7 @@ STREAMS = {
     "tokens": 12,
     "plant_pick": 13,
     "E": 14,
+    "head_logits": 15,
 }
 
 _U64 = np.uint64
