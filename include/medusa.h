@@ -198,8 +198,8 @@ MD_API md_status md_medusa_heads_sampled(const md_bf16* h, const md_bf16* W1, co
                                          const float* uniforms, int32_t* topk_ids, float* topk_keys, float* logits,
                                          void* ws, size_t ws_bytes, void* stream);
 
-/* Size of the library-owned scratch behind md_medusa_heads_static (8 MiB). */
-#define MD_HEADS_STATIC_SCRATCH_BYTES (8u << 20)
+/* Size of the library-owned scratch behind md_medusa_heads_static (32 MiB). */
+#define MD_HEADS_STATIC_SCRATCH_BYTES (32u << 20)
 
 /* md_medusa_heads for callers that cannot allocate device memory.
  * (An addition of this library: the pages have no counterpart.)

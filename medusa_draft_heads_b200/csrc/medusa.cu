@@ -13,6 +13,7 @@
 #include "heads.cuh"
 #include "heads_gemm.cuh"
 #include "heads_gemm2.cuh"
+#include "heads_skinny.cuh"
 #include "tree_build.cuh"
 #include "attention.cuh"
 #include "attention_tc.cuh"
@@ -346,6 +347,101 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   ma.partitioned = 1; ma.units = K * pl.ntiles2; ma.ntiles = pl.ntiles2; ma.kh = K;
   ma.stages = 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
+  return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
+}
+
+// ---------------- tensor-core heads with the weights as M (5 .. 64 rows) ----------------
+// Workspace: z [K, NR, d] bf16, two partial-sum slots per CTA, one ticket per
+// unit of both phases, and the phase-2 candidates [M, K, G2, kmax].
+struct SkinnyPlan {
+  int NR;                  // rows padded to 16, 32 or 64 (the MMA's N)
+  int S, nt1, nt2;         // stages per unit, column tiles of phase 1 (d) and phase 2 (V)
+  int G1, G2;              // CTAs of the two phases
+  size_t off_z, off_part, off_tick, off_cval, off_cid, bytes;
+};
+
+inline bool skinny_rows(int M) { return M >= md::skinny::kMinRows && M <= md::skinny::kMaxRows; }
+
+SkinnyPlan skinny_plan(int M, int d, int V, int K, int kmax) {
+  using md::heads::align256;
+  SkinnyPlan p;
+  p.NR = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.S = d / md::skinny::kBK;
+  p.nt1 = (d + md::skinny::kTile - 1) / md::skinny::kTile;
+  p.nt2 = (V + md::skinny::kTile - 1) / md::skinny::kTile;
+  p.G1 = int(std::min<long long>(num_sms(), (long long)K * p.nt1 * p.S));
+  p.G2 = int(std::min<long long>(num_sms(), (long long)K * p.nt2 * p.S));
+  size_t o = 0;
+  p.off_z = o;    o = align256(o + size_t(K) * p.NR * d * 2);
+  p.off_part = o; o = align256(o + size_t(std::max(p.G1, p.G2)) * 2 * M * md::skinny::kTile * 4);
+  p.off_tick = o; o = align256(o + size_t(K) * (p.nt1 + p.nt2) * 4);
+  p.off_cval = o; o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
+  p.off_cid = o;  o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
+  p.bytes = o;
+  return p;
+}
+
+template <int EPI, int NR>
+md_status launch_skinny(const CUtensorMap& wmap, const CUtensorMap& xmap, const md::skinny::Args& a, int grid,
+                        bool pdl, cudaStream_t st) {
+  auto kern = md::skinny::heads_skinny_kernel<EPI, NR>;
+  const int smem = md::skinny::Cfg<NR>::kSmem;
+  md_status s;
+  if ((s = set_smem(kern, smem)) != MD_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(md::skinny::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, kern, wmap, xmap, a));
+}
+
+template <int NR>
+md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, int kmax, const md_bf16* h,
+                              const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, const int32_t* kph,
+                              int32_t* topk_ids, float* topk_vals, float* logits_dbg, const float* gumbel_u,
+                              float inv_tau, uint8_t* ws, cudaStream_t st) {
+  using namespace md::skinny;
+  md_status s;
+  Args a = {};
+  a.M = M; a.d = d; a.Kh = K; a.S = pl.S; a.kmax = kmax; a.kh = 0;
+  a.h = h; a.b1 = b1;
+  a.z = reinterpret_cast<uint16_t*>(ws + pl.off_z);
+  a.NRz = NR; a.zg_mk = 0;
+  a.part = reinterpret_cast<float*>(ws + pl.off_part);
+  int* tick = reinterpret_cast<int*>(ws + pl.off_tick);
+  for (int k = 0; k < MD_MAX_K; ++k) a.kph[k] = k < K ? kph[k] : 0;
+  if ((s = cuda_ok(cudaMemsetAsync(tick, 0, size_t(K) * (pl.nt1 + pl.nt2) * 4, st))) != MD_OK) return s;
+
+  // phase 1: z = bf16(h + SiLU(h W1_k + b1_k)) -- W1_k^T as the MMA's A, h^T as its B
+  CUtensorMap wmap, xmap;
+  if ((s = make_map_3d_sw128(&wmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&xmap, h, d, M, 1, kBK, NR)) != MD_OK) return s;
+  a.N = d; a.ntiles = pl.nt1; a.tickets = tick;
+  if ((s = launch_skinny<EPI_SILU, NR>(wmap, xmap, a, pl.G1, false, st)) != MD_OK) return s;
+
+  // phase 2: logits = z_k Wv_k, running top-k per (row, head, CTA)
+  if ((s = make_map_3d_sw128(&wmap, Wv, V, d, K, 64, kBK)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&xmap, a.z, d, NR, K, kBK, NR)) != MD_OK) return s;
+  a.N = V; a.ntiles = pl.nt2; a.tickets = tick + size_t(K) * pl.nt1;
+  a.cand_val = reinterpret_cast<float*>(ws + pl.off_cval);
+  a.cand_id = reinterpret_cast<int*>(ws + pl.off_cid);
+  a.logits_dbg = logits_dbg; a.gumbel_u = gumbel_u; a.inv_tau = inv_tau;
+  if ((s = launch_skinny<EPI_TOPK, NR>(wmap, xmap, a, pl.G2, true, st)) != MD_OK) return s;
+
+  // phase 3: merge the CTAs' lists
+  md::heads::MergeArgs ma;
+  ma.cand_val = a.cand_val; ma.cand_id = a.cand_id;
+  ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
+  ma.K = K; ma.kmax = kmax; ma.nslots = pl.G2;
+  ma.partitioned = 1; ma.units = K * pl.nt2; ma.ntiles = pl.nt2; ma.kh = K;
+  ma.stages = pl.S;
+  for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = a.kph[k];
   return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
 }
 
@@ -691,6 +787,20 @@ md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, con
     return MD_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
+  if (M > md::heads::kMaxM && skinny_rows(M)) {
+    // tensor cores with the weights as M: h, W1, Wv feed TMA directly
+    if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
+    const SkinnyPlan pl = skinny_plan(M, d, V, K, kmax);
+    if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
+    if (pl.NR == 16)
+      return launch_heads_skinny<16>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
+                                     logits_dbg, gumbel_u, inv_tau, w, st);
+    if (pl.NR == 32)
+      return launch_heads_skinny<32>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
+                                     logits_dbg, gumbel_u, inv_tau, w, st);
+    return launch_heads_skinny<64>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
+                                   logits_dbg, gumbel_u, inv_tau, w, st);
+  }
   if (M > md::heads::kMaxM) {
     // tensor-core path: h, W1, Wv feed TMA directly (16-byte aligned rows: d % 64, V % 8)
     if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
@@ -807,7 +917,8 @@ md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t
   md_status s = heads_check(M, d, V, K, kmax);
   if (s != MD_OK) return s;
   *bytes = M <= md::heads::kMaxM ? md::heads::make_plan(M, d, V, K, kmax, num_sms()).bytes
-                                  : gemm_plan(M, d, V, K, kmax).bytes;
+           : skinny_rows(M)        ? skinny_plan(M, d, V, K, kmax).bytes
+                                   : gemm_plan(M, d, V, K, kmax).bytes;
   return MD_OK;
 }
 

@@ -110,7 +110,7 @@ def test_static_heads_checks_arguments_before_scratch_size(libmedusa):
     fn.restype = I
     kph = _i32([10, 10, 10, 10])
     fake = ctypes.c_void_p(4096)          # never dereferenced: the call returns before any launch
-    big = (128, 8192, 128256, 4)          # scratch far beyond the 8 MiB array
+    big = (1024, 8192, 128256, 4)         # scratch far beyond the 32 MiB array
     assert fn(None, fake, fake, fake, *big, kph, 10, fake, fake, None, None) == -1
     assert fn(fake, fake, fake, fake, *big, None, 10, fake, fake, None, None) == -1
     assert fn(fake, fake, fake, fake, *big, _i32([10, 10, 11, 10]), 10, fake, fake, None, None) == -1

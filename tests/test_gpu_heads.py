@@ -131,6 +131,31 @@ def test_tensor_core_fused_equals_debug_run():
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+# ------------- tensor cores with the weights as the MMA's M (5 .. 64 rows) -------------
+
+@pytest.mark.parametrize("M,d,V,kph", [
+    (5, 1024, 8192, (10,)),                  # one head: 4 phase-1 units over 64 CTAs, 16 parts each
+    (10, 4096, 4096, (10,)),                 # a Hydra level's row count; units cut into many parts
+    (16, 576, 3000, (4, 3, 2, 2)),           # 9 stages per unit, ragged last vocabulary tile
+    (33, 512, 1000, (10, 10, 10, 10)),       # 64-row padding, 33 live rows
+    (64, 256, 2056, (16, 1, 7, 3)),          # the largest row count of this path
+    (100, 256, 1024, (10, 10, 10, 10)),      # 65 .. 128 rows: one 128-row tile per CTA
+])
+def test_weights_as_m_heads_match_oracle(M, d, V, kph):
+    h, W1, b1, Wv = head_weights(500 + M, d, V, len(kph), M)
+    ids, vals, logits = _run(h, W1, b1, Wv, kph)
+    ids2, vals2, logits2 = _run(h, W1, b1, Wv, kph)
+    # the parts of a cut unit are summed in a fixed order: runs agree bit for bit
+    assert np.array_equal(logits, logits2) and np.array_equal(ids, ids2) and np.array_equal(vals, vals2)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph)
+    err = normwise(logits, rlog)
+    assert err.max() <= HEADS_RTOL, err.max()
+    assert np.median(err) <= 1e-5, np.median(err)
+    for m in range(M):
+        for k, kk in enumerate(kph):
+            check_topk_row(ids[m, k], vals[m, k], rlog[m, k], kk)
+
+
 # ------------------------- shared vocabulary projection -------------------------
 
 def _run_shared(h, W1, b1, Wv, kph, kmax=None):

@@ -21,6 +21,8 @@ import medusa_draft_heads_b200 as md
 
 from .helpers import head_weights, bf16_tensor
 
+STATIC_BYTES = 32 << 20     # MD_HEADS_STATIC_SCRATCH_BYTES in include/medusa.h
+
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +50,7 @@ def _call_static(h, W1, b1, Wv, kph, ids, vals, logits=None):
 def test_static_scratch_matches_workspace_call(M, d, V, kph):
     h, W1, b1, Wv = (bf16_tensor(x) for x in head_weights(900 + M, d, V, len(kph), M))
     K, kmax = len(kph), max(kph)
-    assert md.heads_workspace_bytes(M, d, V, K, kmax) <= (8 << 20)
+    assert md.heads_workspace_bytes(M, d, V, K, kmax) <= STATIC_BYTES
     ref_ids = torch.empty((M, K, kmax), dtype=torch.int32, device="cuda")
     ref_vals = torch.empty((M, K, kmax), dtype=torch.float32, device="cuda")
     ws = md.workspace(md.heads_workspace_bytes(M, d, V, K, kmax))
@@ -65,9 +67,9 @@ def test_static_scratch_matches_workspace_call(M, d, V, kph):
 
 
 def test_static_scratch_refuses_oversized_shapes():
-    """M = 128 rows of 70B-shaped heads need more scratch than the array holds."""
-    M, d, V, K, kmax = 128, 8192, 128256, 4, 10
-    assert md.heads_workspace_bytes(M, d, V, K, kmax) > (8 << 20)
+    """M = 1024 rows of 70B-shaped heads need more scratch than the array holds."""
+    M, d, V, K, kmax = 1024, 8192, 128256, 4, 10
+    assert md.heads_workspace_bytes(M, d, V, K, kmax) > STATIC_BYTES
     h = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
     W1 = torch.empty((K, d, d), dtype=torch.bfloat16, device="cuda")
     b1 = torch.empty((K, d), dtype=torch.bfloat16, device="cuda")
