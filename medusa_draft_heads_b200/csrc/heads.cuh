@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kW1Threads, w1_blocks_per_sm(M)) heads_w1_kern
   __shared__ int is_last;
 
   pdl_launch_dependents();
+  pdl_wait_primary();   // h and the counters may come from the work before (dependent launch)
 
   const int k = blockIdx.z, s = blockIdx.y, ct = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,32 +308,39 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
     if (lane == 0) {
       prefetch_tensormap(&wv_map);
       const uint64_t pol = policy_evict_first();
-      bool waited_primary = false;
-      int it = 0;
-      bool ok = true;
       long long i0, i1;                    // this CTA's (unit, stage) items
       item_range(a, stages_per_unit, i0, i1);
-      for (long long w = i0; w < i1 && ok; ++w, ++it) {
+      auto load_w = [&](long long w, int slot) {
         const int unit = int(w / stages_per_unit), s = int(w % stages_per_unit);
         const int k = unit / a.ntiles, tile = unit % a.ntiles;
-        {
-          const int slot = it % ns;
-          if (it >= ns && !mbar_wait(smem_u32(&empty[slot]), ((it / ns) - 1) & 1)) {
-            set_status(MD_DEV_TIMEOUT);
-            ok = false;
-            break;
-          }
-          const uint32_t fb = smem_u32(&full[slot]);
-          mbar_arrive_expect_tx(fb, kStageWBytes + kStageZBytes);
-          tma_load_2d_hint(smem_u32(stage_w + size_t(slot) * kStageWBytes), &wv_map, tile * kTileV,
-                           k * a.d + s * kStageRows, fb, pol);
-          if (!waited_primary) {  // z comes from phase 1: wait for it only now
-            pdl_wait_primary();
-            waited_primary = true;
-          }
-          bulk_load(smem_u32(stage_z + size_t(slot) * kStageZBytes),
-                    a.zt + (size_t(k) * a.d + size_t(s) * kStageRows) * kZPad, kStageZBytes, fb);
+        tma_load_2d_hint(smem_u32(stage_w + size_t(slot) * kStageWBytes), &wv_map, tile * kTileV,
+                         k * a.d + s * kStageRows, smem_u32(&full[slot]), pol);
+      };
+      auto load_z = [&](long long w, int slot) {
+        const int unit = int(w / stages_per_unit), s = int(w % stages_per_unit);
+        const int k = unit / a.ntiles;
+        bulk_load(smem_u32(stage_z + size_t(slot) * kStageZBytes),
+                  a.zt + (size_t(k) * a.d + size_t(s) * kStageRows) * kZPad, kStageZBytes, smem_u32(&full[slot]));
+      };
+      // The first stages' weights do not depend on phase 1: request them
+      // before waiting for it; z (phase 1's output) only after.
+      const int pre = int(min((long long)ns, i1 - i0));
+      for (int j = 0; j < pre; ++j) {
+        mbar_arrive_expect_tx(smem_u32(&full[j]), kStageWBytes + kStageZBytes);
+        load_w(i0 + j, j);
+      }
+      pdl_wait_primary();
+      for (int j = 0; j < pre; ++j) load_z(i0 + j, j);
+      int it = pre;
+      for (long long w = i0 + pre; w < i1; ++w, ++it) {
+        const int slot = it % ns;
+        if (!mbar_wait(smem_u32(&empty[slot]), ((it / ns) - 1) & 1)) {
+          set_status(MD_DEV_TIMEOUT);
+          break;
         }
+        mbar_arrive_expect_tx(smem_u32(&full[slot]), kStageWBytes + kStageZBytes);
+        load_w(w, slot);
+        load_z(w, slot);
       }
       // Drain: wait until the consumers have released every issued stage so
       // no copy is in flight into shared memory when the CTA exits.
@@ -600,15 +608,14 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
   // entries; only those entries are sorted.
   __shared__ float red_v[kMergeThreads / 32];
   __shared__ int red_i[kMergeThreads / 32];
-  __shared__ int n_keep;
   {
     float bv = -INFINITY;
     int bi = INT_MAX;
     for (int l = threadIdx.x; l < n_lists; l += kMergeThreads) {
       const size_t at = base + size_t(slot_of[l]) * a.kmax + (kk - 1);
       const int x = a.cand_id[at];
+      const float v = a.cand_val[at];
       if (x >= 0) {
-        const float v = a.cand_val[at];
         if (better(v, x, bv, bi)) {
           bv = v;
           bi = x;
@@ -628,7 +635,6 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
       red_v[warp] = bv;
       red_i[warp] = bi;
     }
-    if (threadIdx.x == 0) n_keep = 0;
     __syncthreads();
   }
   float tv = red_v[0];
@@ -640,36 +646,48 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
       ti = red_i[w];
     }
 
-  // 3. gather the (value, id) pairs at or above the threshold, in slot order
+  // 3. gather the (value, id) pairs at or above the threshold, in slot order;
+  // every candidate this thread looks at is loaded first, so the loads are in
+  // flight together instead of one dependent round trip per pass
+  constexpr int kPer = kMergeCap / kMergeThreads;
   const int n = n_lists * kk;
-  for (int e0 = 0; e0 < n; e0 += kMergeThreads) {
-    const int e = e0 + threadIdx.x;
-    float v = -INFINITY;
-    int id = -1;
+  float cv[kPer];
+  int ci[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int e = q * kMergeThreads + threadIdx.x;
+    cv[q] = -INFINITY;
+    ci[q] = -1;
     if (e < n) {
       const size_t at = base + size_t(slot_of[e / kk]) * a.kmax + e % kk;
-      id = a.cand_id[at];
-      if (id >= 0) v = a.cand_val[at];
+      ci[q] = a.cand_id[at];
+      cv[q] = a.cand_val[at];
     }
-    const bool keep = id >= 0 && (better(v, id, tv, ti) || (v == tv && id == ti));
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) warp_cnt[warp] = __popc(bal);
-    __syncthreads();
-    int off = n_keep;
-    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
-    if (keep) {
-      sv[off + __popc(bal & ((1u << lane) - 1))] = v;
-      si[off + __popc(bal & ((1u << lane) - 1))] = id;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int t = n_keep;
-      for (int w = 0; w < kMergeThreads / 32; ++w) t += warp_cnt[w];
-      n_keep = t;
-    }
-    __syncthreads();
   }
-  const int nk = n_keep;
+  // keep flags and per-warp counts of every pass, then one prefix: the order
+  // of the kept entries is the candidates' order e = q * threads + thread
+  __shared__ int pass_cnt[kPer][kMergeThreads / 32];
+  unsigned bal[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const bool keep = ci[q] >= 0 && (better(cv[q], ci[q], tv, ti) || (cv[q] == tv && ci[q] == ti));
+    bal[q] = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) pass_cnt[q][warp] = __popc(bal[q]);
+  }
+  __syncthreads();
+  int run = 0;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    int off = run;
+    for (int w = 0; w < warp; ++w) off += pass_cnt[q][w];
+    if ((bal[q] >> lane) & 1u) {
+      const int at = off + __popc(bal[q] & ((1u << lane) - 1));
+      sv[at] = cv[q];
+      si[at] = ci[q];
+    }
+    for (int w = 0; w < kMergeThreads / 32; ++w) run += pass_cnt[q][w];
+  }
+  const int nk = run;
   int N = 32;
   while (N < nk) N <<= 1;
   for (int e = nk + threadIdx.x; e < N; e += kMergeThreads) {   // pad with (-inf, INT_MAX)

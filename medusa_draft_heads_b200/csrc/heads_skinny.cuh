@@ -1,4 +1,4 @@
-// Medusa draft heads on the tensor cores for a few hidden rows (5 .. 64),
+// Medusa draft heads on the tensor cores for a few hidden rows (2 .. 64),
 // with the weights on the MMA's M side.
 //
 // Source: "Medusa heads versus separate draft model", sections "What each one
@@ -8,8 +8,8 @@
 //   phase 2  logits = z_k Wv_k (d x V), each row's top-k (or Gumbel top-k)
 //
 // With a handful of rows the call is still a weight stream: every weight byte
-// is used M times. On CUDA cores M FMAs per weight element outrun the
-// stream's time from about 5 rows, and a 128-row MMA tile pads M to 128. Here
+// is used M times. On CUDA cores the M FMAs per weight element slow the stream
+// from two rows on, and a 128-row MMA tile pads M to 128. Here
 // the product is computed transposed, D^T = W^T x^T: 128 output columns of the
 // weights form the MMA's M (the weight tile is N-major as TMA brings it from
 // the input-major matrix) and the rows form its N (NR = 16, 32 or 64, rows
@@ -45,7 +45,7 @@ constexpr uint32_t kWBox = 64 * kBK * 2;     // 8 KB: 64 reduction rows x 64 col
 constexpr uint32_t kWBytes = 4 * kWBox;      // 32 KB per stage
 constexpr int kThreads = 192;
 constexpr int kChunk = 16;                   // rows per tcgen05.ld in the epilogue
-constexpr int kMinRows = 5, kMaxRows = 64;   // the launcher's range of rows for this path
+constexpr int kMinRows = 2, kMaxRows = 64;   // the launcher's range of rows for this path
 
 enum { EPI_SILU = 0, EPI_TOPK = 1 };
 

@@ -122,10 +122,13 @@ md_status set_smem(Kernel k, int bytes) {
 
 // ----------------------------- heads launchers -----------------------------
 
+// zeroed: the workspace's counters and tickets are already zero (cleared by
+// the caller earlier on the stream), so no memset separates this call from
+// the kernel before it and the first kernel is launched dependent on it.
 template <int M>
 md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
                        const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
-                       const float* gumbel_u, float inv_tau, uint8_t* ws, cudaStream_t st) {
+                       const float* gumbel_u, float inv_tau, uint8_t* ws, cudaStream_t st, bool zeroed = false) {
   using namespace md::heads;
   md_status s;
   // phase 1
@@ -137,11 +140,17 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   wa.d = pl.d; wa.K = pl.K; wa.splits = pl.splits; wa.rows = pl.rows; wa.ntile_o = pl.ntile_o;
   wa.shared = 0;
   // phase-1 counters and phase-2 tickets are contiguous: one memset
-  if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, pl.off_spart - pl.off_cnt, st))) != MD_OK) return s;
+  if (!zeroed && (s = cuda_ok(cudaMemsetAsync(wa.counters, 0, pl.off_spart - pl.off_cnt, st))) != MD_OK) return s;
   const int w1_smem = pl.rows * 16 + kConsumerWarps * M * kW1TileO * 4;
   if ((s = set_smem(heads_w1_kernel<M>, w1_smem)) != MD_OK) return s;
-  heads_w1_kernel<M><<<dim3(pl.ntile_o, pl.splits, pl.K), kW1Threads, w1_smem, st>>>(wa);
-  if ((s = last_launch()) != MD_OK) return s;
+  if (zeroed) {
+    if ((s = launch_pdl(heads_w1_kernel<M>, dim3(pl.ntile_o, pl.splits, pl.K), dim3(kW1Threads), w1_smem, st,
+                        wa)) != MD_OK)
+      return s;
+  } else {
+    heads_w1_kernel<M><<<dim3(pl.ntile_o, pl.splits, pl.K), kW1Threads, w1_smem, st>>>(wa);
+    if ((s = last_launch()) != MD_OK) return s;
+  }
 
   // phase 2 (programmatic dependent launch: its TMA of Wv may start before phase 1 ends)
   CUtensorMap map;
@@ -362,6 +371,10 @@ struct SkinnyPlan {
 
 inline bool skinny_rows(int M) { return M >= md::skinny::kMinRows && M <= md::skinny::kMaxRows; }
 
+// The CUDA-core stream serves one row; from two rows the tensor cores (its
+// FMA work grows with M: 1.50 vs 1.32 ms at two rows of 70B heads).
+inline bool stream_rows(int M) { return M < md::skinny::kMinRows; }
+
 SkinnyPlan skinny_plan(int M, int d, int V, int K, int kmax) {
   using md::heads::align256;
   SkinnyPlan p;
@@ -405,7 +418,7 @@ template <int NR>
 md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, int kmax, const md_bf16* h,
                               const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, const int32_t* kph,
                               int32_t* topk_ids, float* topk_vals, float* logits_dbg, const float* gumbel_u,
-                              float inv_tau, uint8_t* ws, cudaStream_t st) {
+                              float inv_tau, uint8_t* ws, cudaStream_t st, bool zeroed = false) {
   using namespace md::skinny;
   md_status s;
   Args a = {};
@@ -416,14 +429,14 @@ md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, 
   a.part = reinterpret_cast<float*>(ws + pl.off_part);
   int* tick = reinterpret_cast<int*>(ws + pl.off_tick);
   for (int k = 0; k < MD_MAX_K; ++k) a.kph[k] = k < K ? kph[k] : 0;
-  if ((s = cuda_ok(cudaMemsetAsync(tick, 0, size_t(K) * (pl.nt1 + pl.nt2) * 4, st))) != MD_OK) return s;
+  if (!zeroed && (s = cuda_ok(cudaMemsetAsync(tick, 0, size_t(K) * (pl.nt1 + pl.nt2) * 4, st))) != MD_OK) return s;
 
   // phase 1: z = bf16(h + SiLU(h W1_k + b1_k)) -- W1_k^T as the MMA's A, h^T as its B
   CUtensorMap wmap, xmap;
   if ((s = make_map_3d_sw128(&wmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&xmap, h, d, M, 1, kBK, NR)) != MD_OK) return s;
   a.N = d; a.ntiles = pl.nt1; a.tickets = tick;
-  if ((s = launch_skinny<EPI_SILU, NR>(wmap, xmap, a, pl.G1, false, st)) != MD_OK) return s;
+  if ((s = launch_skinny<EPI_SILU, NR>(wmap, xmap, a, pl.G1, zeroed, st)) != MD_OK) return s;
 
   // phase 2: logits = z_k Wv_k, running top-k per (row, head, CTA)
   if ((s = make_map_3d_sw128(&wmap, Wv, V, d, K, 64, kBK)) != MD_OK) return s;
@@ -450,18 +463,40 @@ md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, 
 // (m, k) -> m*K + k as rows of one head against the single projection.
 
 struct SharedPlan {
-  bool stream;                 // M*K <= 4: CUDA-core weight stream; else tensor cores
+  bool stream;                 // M*K == 1: CUDA-core weight stream
+  bool skinny;                 // 2 <= M*K <= 64: tensor cores with the weights as M; else row-tile GEMMs
   md::heads::Plan p1, p2;      // streaming: phase-1 plan (M rows, K heads), phase-2 plan (M*K rows, 1 head)
   GemmPlan g1, g2;             // tensor cores: phase 1 (M rows, K heads), phase 2 (M*K rows, 1 head)
   size_t off2, bytes;
   size_t tick2, spart2, cval2, cid2;   // streaming: phase-2 tickets, partials, candidates (from off2)
+  // weights as M: rows padded to NR1 (phase 1, M) and NR2 (phase 2, M*K)
+  int NR1, NR2, S, nt1, nt2, G1, G2;
+  size_t off_z, off_part, off_tick, off_cval, off_cid;
 };
+
+inline int skinny_pad(int rows) { return rows <= 16 ? 16 : (rows <= 32 ? 32 : 64); }
 
 SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
   using md::heads::align256;
   SharedPlan p{};
-  p.stream = M * K <= md::heads::kMaxM;
-  if (p.stream) {
+  p.stream = M * K == 1;
+  p.skinny = !p.stream && skinny_rows(M * K);
+  if (p.skinny) {
+    p.NR1 = skinny_pad(M);
+    p.NR2 = skinny_pad(M * K);
+    p.S = d / md::skinny::kBK;
+    p.nt1 = (d + md::skinny::kTile - 1) / md::skinny::kTile;
+    p.nt2 = (V + md::skinny::kTile - 1) / md::skinny::kTile;
+    p.G1 = int(std::min<long long>(num_sms(), (long long)K * p.nt1 * p.S));
+    p.G2 = int(std::min<long long>(num_sms(), (long long)p.nt2 * p.S));
+    size_t o = 0;
+    p.off_z = o;    o = align256(o + size_t(p.NR2) * d * 2);
+    p.off_part = o; o = align256(o + size_t(std::max(p.G1, p.G2)) * 2 * (M * K) * md::skinny::kTile * 4);
+    p.off_tick = o; o = align256(o + size_t(K * p.nt1 + p.nt2) * 4);
+    p.off_cval = o; o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
+    p.off_cid = o;  o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
+    p.bytes = o;
+  } else if (p.stream) {
     p.p1 = md::heads::make_plan(M, d, V, K, kmax, num_sms());
     p.p2 = md::heads::make_plan(M * K, d, V, 1, kmax, num_sms());
     p.off2 = align256(p.p1.off_cval);                    // phase-2 data after phase-1 data
@@ -477,6 +512,52 @@ SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
     p.bytes = p.off2 + (p.g2.bytes - p.g2.off_cval);
   }
   return p;
+}
+
+// One projection for all heads on the tensor cores with the weights as M:
+// phase 1 is the K heads' residual blocks on the M rows (z row (m, k) written
+// to row m*K + k), phase 2 one head over the M*K rows, row m*K + k keeping
+// head k's top-k size.
+template <int NR1, int NR2>
+md_status launch_heads_shared_skinny(const SharedPlan& sp, int M, int d, int V, int K, int kmax, const md_bf16* h,
+                                     const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, const int32_t* kph,
+                                     int32_t* topk_ids, float* topk_vals, float* logits_dbg, uint8_t* ws,
+                                     cudaStream_t st) {
+  using namespace md::skinny;
+  md_status s;
+  Args a = {};
+  a.d = d; a.S = sp.S; a.kmax = kmax;
+  a.h = h; a.b1 = b1;
+  a.z = reinterpret_cast<uint16_t*>(ws + sp.off_z);
+  a.NRz = NR2; a.zg_mk = 1;
+  a.part = reinterpret_cast<float*>(ws + sp.off_part);
+  int* tick = reinterpret_cast<int*>(ws + sp.off_tick);
+  for (int k = 0; k < MD_MAX_K; ++k) a.kph[k] = k < K ? kph[k] : 0;
+  if ((s = cuda_ok(cudaMemsetAsync(tick, 0, size_t(K * sp.nt1 + sp.nt2) * 4, st))) != MD_OK) return s;
+
+  CUtensorMap wmap, xmap;
+  if ((s = make_map_3d_sw128(&wmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&xmap, h, d, M, 1, kBK, NR1)) != MD_OK) return s;
+  a.M = M; a.Kh = K; a.N = d; a.ntiles = sp.nt1; a.tickets = tick; a.kh = 0;
+  if ((s = launch_skinny<EPI_SILU, NR1>(wmap, xmap, a, sp.G1, false, st)) != MD_OK) return s;
+
+  if ((s = make_map_3d_sw128(&wmap, Wv, V, d, 1, 64, kBK)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&xmap, a.z, d, NR2, 1, kBK, NR2)) != MD_OK) return s;
+  a.M = M * K; a.Kh = 1; a.N = V; a.ntiles = sp.nt2; a.tickets = tick + size_t(K) * sp.nt1; a.kh = K;
+  a.zg_mk = 0;
+  a.cand_val = reinterpret_cast<float*>(ws + sp.off_cval);
+  a.cand_id = reinterpret_cast<int*>(ws + sp.off_cid);
+  a.logits_dbg = logits_dbg; a.gumbel_u = nullptr; a.inv_tau = 1.f;
+  if ((s = launch_skinny<EPI_TOPK, NR2>(wmap, xmap, a, sp.G2, true, st)) != MD_OK) return s;
+
+  md::heads::MergeArgs ma;
+  ma.cand_val = a.cand_val; ma.cand_id = a.cand_id;
+  ma.topk_ids = topk_ids; ma.topk_vals = topk_vals;
+  ma.K = 1; ma.kmax = kmax; ma.nslots = sp.G2;
+  ma.partitioned = 1; ma.units = sp.nt2; ma.ntiles = sp.nt2; ma.kh = K;
+  ma.stages = sp.S;
+  for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = a.kph[k];
+  return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
 }
 
 template <int MK>
@@ -727,8 +808,9 @@ struct HydraPlan {
   int rows;                           // top-k rows of all levels
   int8_t slot[MD_MAX_T];              // node -> index among its depth's nodes with children (-1: none)
   int8_t node[MD_MAX_K][MD_MAX_T];    // level l, index q -> node
-  size_t heads_bytes;                 // largest heads workspace of one level
-  size_t off_x, off_ids, off_vals, off_heads, bytes;
+  size_t heads_bytes[MD_MAX_K];       // heads workspace of each level (its own region: the
+  size_t off_heads[MD_MAX_K];         // counters of every level are cleared once, up front)
+  size_t off_x, off_ids, off_vals, bytes;
 };
 
 md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPlan* out) {
@@ -749,7 +831,6 @@ md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPl
   md_status s = heads_check(1, d, V, 1, kmax);
   if (s != MD_OK) return s;
   int rows = 0, maxn = 1;
-  p.heads_bytes = 0;
   for (int l = 0; l < p.L; ++l) {
     p.row0[l] = rows;
     rows += B * p.n[l];
@@ -757,26 +838,46 @@ md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPl
     if (tree->kph[l] > kmax) return MD_ERR_INVALID_ARG;
     size_t hb = 0;
     if ((s = md_heads_workspace(B * p.n[l], d, V, 1, kmax, &hb)) != MD_OK) return s;
-    p.heads_bytes = std::max(p.heads_bytes, hb);
+    p.heads_bytes[l] = hb;
   }
   p.rows = rows;
   size_t o = 0;
   p.off_x = o;     o = align256(o + size_t(B) * maxn * d * 2);
   p.off_ids = o;   o = align256(o + size_t(std::max(rows, 1)) * kmax * 4);
   p.off_vals = o;  o = align256(o + size_t(std::max(rows, 1)) * kmax * 4);
-  p.off_heads = o; o = align256(o + p.heads_bytes);
+  for (int l = 0; l < p.L; ++l) {
+    p.off_heads[l] = o;
+    o = align256(o + p.heads_bytes[l]);
+  }
   p.bytes = o;
   *out = p;
   return MD_OK;
 }
 
+// The workspace ranges a heads call needs zero at its start (counters and
+// tickets), as [offset, offset + bytes); bytes = 0 when there are none.
+void heads_zero_range(int M, int d, int V, int K, int kmax, size_t* off, size_t* bytes) {
+  *off = 0;
+  *bytes = 0;
+  if (stream_rows(M)) {
+    const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
+    *off = pl.off_cnt;
+    *bytes = pl.off_spart - pl.off_cnt;
+  } else if (skinny_rows(M)) {
+    const SkinnyPlan pl = skinny_plan(M, d, V, K, kmax);
+    *off = pl.off_tick;
+    *bytes = size_t(K) * (pl.nt1 + pl.nt2) * 4;
+  }
+}
+
 // md_medusa_heads and md_medusa_heads_sampled: checks, then the streaming
-// (M <= 4) or tensor-core path. gumbel_u null: top-k of the logits; else the
-// top-k of the Gumbel keys logit * inv_tau - ln(-ln u).
+// (one row), weights-as-M (2 .. 64 rows) or row-tile tensor-core path.
+// gumbel_u null: top-k of the logits; else the top-k of the Gumbel keys
+// logit * inv_tau - ln(-ln u). zeroed: heads_zero_range is already zero.
 md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, int32_t M,
                      int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax, int32_t* topk_ids,
                      float* topk_vals, float* logits_dbg, const float* gumbel_u, float inv_tau, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     size_t ws_bytes, void* stream, bool zeroed = false) {
   if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
   md_status s = heads_check(M, d, V, K, kmax);
   if (s != MD_OK) return s;
@@ -787,21 +888,21 @@ md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, con
     return MD_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
-  if (M > md::heads::kMaxM && skinny_rows(M)) {
+  if (skinny_rows(M)) {
     // tensor cores with the weights as M: h, W1, Wv feed TMA directly
     if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
     const SkinnyPlan pl = skinny_plan(M, d, V, K, kmax);
     if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
     if (pl.NR == 16)
       return launch_heads_skinny<16>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
-                                     logits_dbg, gumbel_u, inv_tau, w, st);
+                                     logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
     if (pl.NR == 32)
       return launch_heads_skinny<32>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
-                                     logits_dbg, gumbel_u, inv_tau, w, st);
+                                     logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
     return launch_heads_skinny<64>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
-                                   logits_dbg, gumbel_u, inv_tau, w, st);
+                                   logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
   }
-  if (M > md::heads::kMaxM) {
+  if (!stream_rows(M)) {
     // tensor-core path: h, W1, Wv feed TMA directly (16-byte aligned rows: d % 64, V % 8)
     if (!aligned(h, 16) || !aligned(b1, 16)) return MD_ERR_INVALID_ARG;
     if (!ws || ws_bytes < gemm_plan(M, d, V, K, kmax).bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
@@ -818,13 +919,9 @@ md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, con
   }
   const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
   if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
-  switch (M) {
-    case 1: return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
-    case 2: return launch_heads<2>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
-    case 3: return launch_heads<3>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
-    case 4: return launch_heads<4>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
-    default: return MD_ERR_UNSUPPORTED;
-  }
+  if (M != 1) return MD_ERR_UNSUPPORTED;
+  return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st,
+                         zeroed);
 }
 
 // Scratch of md_medusa_heads_static: a fixed array in the library's device
@@ -916,9 +1013,9 @@ md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, int32_t
   if (!bytes) return MD_ERR_INVALID_ARG;
   md_status s = heads_check(M, d, V, K, kmax);
   if (s != MD_OK) return s;
-  *bytes = M <= md::heads::kMaxM ? md::heads::make_plan(M, d, V, K, kmax, num_sms()).bytes
-           : skinny_rows(M)        ? skinny_plan(M, d, V, K, kmax).bytes
-                                   : gemm_plan(M, d, V, K, kmax).bytes;
+  *bytes = stream_rows(M)   ? md::heads::make_plan(M, d, V, K, kmax, num_sms()).bytes
+           : skinny_rows(M) ? skinny_plan(M, d, V, K, kmax).bytes
+                            : gemm_plan(M, d, V, K, kmax).bytes;
   return MD_OK;
 }
 
@@ -970,15 +1067,22 @@ md_status md_medusa_heads_shared(const md_bf16* h, const md_bf16* W1, const md_b
   const SharedPlan sp = shared_plan(M, d, V, K, kmax);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
-  if (sp.stream) {
-    switch (M * K) {
-      case 1: return launch_heads_shared_stream<1>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-      case 2: return launch_heads_shared_stream<2>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-      case 3: return launch_heads_shared_stream<3>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-      case 4: return launch_heads_shared_stream<4>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
-      default: return MD_ERR_UNSUPPORTED;
-    }
+  if (sp.skinny) {
+#define MD_SHARED_SKINNY(a, b)                                                                                   \
+  if (sp.NR1 == a && sp.NR2 == b)                                                                                \
+    return launch_heads_shared_skinny<a, b>(sp, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, \
+                                            logits_dbg, w, st);
+    MD_SHARED_SKINNY(16, 16)
+    MD_SHARED_SKINNY(16, 32)
+    MD_SHARED_SKINNY(16, 64)
+    MD_SHARED_SKINNY(32, 32)
+    MD_SHARED_SKINNY(32, 64)
+    MD_SHARED_SKINNY(64, 64)
+#undef MD_SHARED_SKINNY
+    return MD_ERR_UNSUPPORTED;
   }
+  if (sp.stream)
+    return launch_heads_shared_stream<1>(sp, M, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
   if (mk <= 4)
     return launch_heads_shared_gemm<4>(sp, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, w, st);
   if (mk <= 8)
@@ -1053,6 +1157,13 @@ md_status md_hydra_draft(const md_tree* tree, const md_bf16* h, int32_t M, const
   uint16_t* x = reinterpret_cast<uint16_t*>(w + p.off_x);
   int32_t* ids = reinterpret_cast<int32_t*>(w + p.off_ids);
   float* vals = reinterpret_cast<float*>(w + p.off_vals);
+  // every level's counters are cleared here, so the levels' kernels follow
+  // one another as dependent launches with no memset between them
+  for (int l = 0; l < p.L; ++l) {
+    size_t zo = 0, zb = 0;
+    heads_zero_range(B * p.n[l], d, V, 1, kmax, &zo, &zb);
+    if (zb && (s = cuda_ok(cudaMemsetAsync(w + p.off_heads[l] + zo, 0, zb, st))) != MD_OK) return s;
+  }
   for (int l = 0; l < p.L; ++l) {
     md::hydra::GatherArgs ga;
     std::memset(&ga, 0, sizeof(ga));
@@ -1070,10 +1181,10 @@ md_status md_hydra_draft(const md_tree* tree, const md_bf16* h, int32_t M, const
                         ga)) != MD_OK)
       return s;
     const size_t r0 = size_t(p.row0[l]);
-    if ((s = md_medusa_heads(x, W1 + size_t(l) * d * d, b1 + size_t(l) * d, Wv + size_t(l) * d * V, B * p.n[l], d, V,
-                             1, &tree->kph[l], kmax, ids + r0 * kmax, vals + r0 * kmax,
-                             logits_dbg ? logits_dbg + r0 * V : nullptr, w + p.off_heads, p.heads_bytes, stream)) !=
-        MD_OK)
+    if ((s = heads_call(x, W1 + size_t(l) * d * d, b1 + size_t(l) * d, Wv + size_t(l) * d * V, B * p.n[l], d, V, 1,
+                        &tree->kph[l], kmax, ids + r0 * kmax, vals + r0 * kmax,
+                        logits_dbg ? logits_dbg + r0 * V : nullptr, nullptr, 1.f, w + p.off_heads[l],
+                        p.heads_bytes[l], stream, true)) != MD_OK)
       return s;
   }
   md::hydra::TokenArgs ta;

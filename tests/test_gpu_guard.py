@@ -57,8 +57,9 @@ def _tree(kph, n):
 
 @pytest.mark.parametrize("M,d,V,kph", [
     (1, 256, 1024, (4, 3, 2, 2)),            # streaming, tiny
-    (3, 320, 1000, (10, 1, 7, 3)),           # streaming, ragged column tile
-    (20, 256, 2056, (16, 16, 16, 16)),       # single-CTA tensor-core GEMM, ragged rows and columns
+    (3, 320, 1000, (10, 1, 7, 3)),           # weights as M, ragged column tile
+    (20, 256, 2056, (16, 16, 16, 16)),       # weights as M, ragged rows and columns
+    (100, 256, 2056, (16, 16, 16, 16)),      # single-CTA row-tile GEMM, ragged rows and columns
     (160, 192, 1288, (10, 10, 10, 10)),      # CTA-pair GEMM, second pair half-empty
 ])
 def test_heads_write_nothing_past_their_buffers(M, d, V, kph):

@@ -96,7 +96,7 @@ def test_heads_reject_bad_arguments():
                         vals, ws)
 
 
-# ------------- tensor-core path (M > 4; CTA pairs once M > 128 rows) -------------
+# ------------- tensor-core paths (M > 1: weights as M up to 64 rows, row tiles up to 128, CTA pairs beyond) -------------
 
 @pytest.mark.parametrize("M,d,V,kph", [(9, 256, 1024, (4, 3, 2, 2)), (40, 320, 1000, (10, 10, 10, 10)),
                                        (130, 512, 2056, (16, 1, 7, 3)), (520, 256, 4096, (10, 10, 10, 10))])
@@ -174,8 +174,10 @@ def _run_shared(h, W1, b1, Wv, kph, kmax=None):
     return ids.cpu().numpy(), vals.cpu().numpy(), logits.cpu().numpy()
 
 
-@pytest.mark.parametrize("M,d,V,kph", [(1, 256, 1024, (4, 3, 2, 2)), (1, 512, 2056, (10, 10, 10, 10)),
+@pytest.mark.parametrize("M,d,V,kph", [(1, 256, 1024, (10,)),                      # one row: streaming
+                                       (1, 256, 1024, (4, 3, 2, 2)), (1, 512, 2056, (10, 10, 10, 10)),
                                        (2, 320, 1000, (16, 1)), (3, 256, 4096, (10, 10, 10, 10)),
+                                       (12, 576, 3000, (16, 7, 3, 1)),             # 48 rows after 12-row phase 1
                                        (130, 256, 1024, (7, 3, 2))])
 def test_shared_projection_matches_oracle(M, d, V, kph):
     K = len(kph)

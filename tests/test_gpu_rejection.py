@@ -33,7 +33,7 @@ def _uniforms(rng, shape):
                                            (20, 256, 4096, (10, 10, 10, 10), 0.7),
                                            (160, 192, 1288, (16, 8, 4, 2), 1.3)])
 def test_sampled_drafts_match_oracle(M, d, V, kph, tau):
-    """Streaming (M <= 4), single-CTA and CTA-pair tensor-core paths: the
+    """Streaming (M = 1), weights-as-M and CTA-pair tensor-core paths: the
     logits equal md_medusa_heads' exactly, and the candidates are the Gumbel
     top-k of the oracle's keys (ids exact where the oracle's neighbouring keys
     are clear of the observed key error)."""

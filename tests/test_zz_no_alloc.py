@@ -6,7 +6,7 @@ never reach the allocator -- so the library offers one variant of the heads
 call whose scratch is a fixed array in its own device image. These checks call
 it through the C ABI (ctypes, raw pointers) twice in a row and compare each
 result with the ordinary md_medusa_heads on the same inputs (streaming,
-single-CTA and CTA-pair tensor-core paths), and check that a shape whose
+weights-as-M, single-CTA and CTA-pair tensor-core paths), and check that a shape whose
 scratch would not fit is refused before anything runs.
 
 This file is named to be collected last, so a run that stops at the first
@@ -46,7 +46,8 @@ def _call_static(h, W1, b1, Wv, kph, ids, vals, logits=None):
 
 
 @pytest.mark.parametrize("M,d,V,kph", [(1, 1024, 8192, (10, 10, 10, 10)), (3, 512, 2056, (16, 1, 7, 3)),
-                                       (20, 256, 4096, (10, 10, 10, 10)), (160, 256, 4096, (10, 10, 10, 10))])
+                                       (20, 256, 4096, (10, 10, 10, 10)), (100, 256, 4096, (10, 10, 10, 10)),
+                                       (160, 256, 4096, (10, 10, 10, 10))])
 def test_static_scratch_matches_workspace_call(M, d, V, kph):
     h, W1, b1, Wv = (bf16_tensor(x) for x in head_weights(900 + M, d, V, len(kph), M))
     K, kmax = len(kph), max(kph)
