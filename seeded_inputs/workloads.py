@@ -77,6 +77,8 @@ BATCHED70B = replace(LLAMA70B, name="llama3-70b-b8", B=8, prefix=(1024, 8192), h
 # Profiling case for the heads kernels: 8B-shaped with a 32000-token vocabulary,
 # so the weights (1.1 GB) exceed L2 while the device footprint stays small.
 PROF_HEADS = replace(LLAMA8B, name="prof-8b-v32000", V=32000)
+# Profiling case for the weights-as-M tensor-core heads: the same weights on 16 rows.
+PROF_SKINNY = replace(PROF_HEADS, name="prof-8b-v32000-b16", B=16)
 # Profiling case for the tensor-core heads: the same weights on 8 x 65 = 520 rows.
 PROF_GEMM = replace(PROF_HEADS, name="prof-8b-v32000-b8", B=8, heads_rows="BT", prefix=(1024, 8192))
 
@@ -90,7 +92,7 @@ LLAMA70B_SAMPLED = replace(LLAMA70B, name="llama3-70b-sampled", mode="sample", t
 # lossless acceptance by rejection sampling (temperature 0.7 for both).
 LLAMA70B_REJECTION = replace(LLAMA70B, name="llama3-70b-rejection", mode="rejection", temperature=0.7)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS, PROF_GEMM,
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA70B, LLAMA70B_CHAIN, BATCHED70B, PROF_HEADS, PROF_SKINNY, PROF_GEMM,
                                  LLAMA70B_SHARED, LLAMA70B_SAMPLED, LLAMA70B_REJECTION)}
 
 

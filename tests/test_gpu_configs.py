@@ -160,7 +160,7 @@ def test_batched_70b_heads_whole_request_and_every_cta():
 
 def test_sweep_8b_heads_b32_single_cta_and_pair_gemm():
     """8B sweep heads at B = 32: the sweep's one hidden row per request
-    (M = 32, single-CTA tcgen05 GEMM), every row checked; and all 32 x 65 tree
+    (M = 32, tcgen05 with the weights as the MMA's M), every row checked; and all 32 x 65 tree
     tokens (M = 2080, CTA-pair GEMM, 17 row tiles in 9 pairs), one row in each
     128-row tile plus the last row."""
     w = sweep_8b(32, "64", 1024)
