@@ -506,6 +506,16 @@ MD_API md_status md_set_wait_limit(uint64_t ns);
  * Errors: MD_ERR_INVALID_ARG (chunk < -1), MD_ERR_CUDA. */
 MD_API md_status md_test_withhold_attention_chunk(int32_t chunk);
 
+/* Diagnostic: reads bytes of device memory once, front to back in 16-byte
+ * non-allocating loads (8 in flight per thread, 4 CTAs of 512 threads per SM),
+ * and folds them into *sink (device, 4 bytes; written only for one particular
+ * XOR value, so that the loads are kept). It measures the read-only bandwidth
+ * that bounds the weight-stream kernels of md_medusa_heads (a copy moves every
+ * byte twice and is not their ceiling). buf 16-byte aligned; bytes a multiple
+ * of 16. Asynchronous on stream.
+ * Errors: MD_ERR_INVALID_ARG (null, misaligned or ragged size), MD_ERR_CUDA. */
+MD_API md_status md_stream_read(const void* buf, size_t bytes, uint32_t* sink, void* stream);
+
 /* Static description of a status code. */
 MD_API const char* md_status_string(md_status status);
 

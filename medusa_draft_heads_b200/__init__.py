@@ -21,5 +21,5 @@ from .binding import (MedusaError, Tree, accept_workspace_bytes, attention_works
                       device_status, heads_shared_workspace_bytes, heads_workspace_bytes, hydra_draft,
                       hydra_logit_rows, hydra_workspace_bytes, lib, medusa_heads, medusa_heads_sampled,
                       medusa_heads_shared, tree_accept, tree_accept_rejection, tree_accept_sampled, tree_attention,
-                      set_wait_limit, tree_build, tree_commit, version, workspace)
+                      set_wait_limit, stream_read, tree_build, tree_commit, version, workspace)
 from .tree_spec import select_tree, tree_arrays  # noqa: F401

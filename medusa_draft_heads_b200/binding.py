@@ -48,6 +48,7 @@ _SIGNATURES = {
     "md_tree_commit": [_P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P],
     "md_get_device_status": [_P, ctypes.POINTER(_I), _I],
     "md_set_wait_limit": [ctypes.c_uint64],
+    "md_stream_read": [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p],
     "md_test_withhold_attention_chunk": [_I],
     "md_status_string": [_I],
     "md_version": [],
@@ -408,6 +409,16 @@ def set_wait_limit(ns: int = 0):
 def withhold_attention_chunk_for_test(chunk: int):
     """md_test_withhold_attention_chunk: the timeout-path test hook (-1 = off)."""
     _check(lib().md_test_withhold_attention_chunk(int(chunk)), "md_test_withhold_attention_chunk")
+
+
+def stream_read(buf, sink, stream=None):
+    """md_stream_read: one read-only pass over a contiguous CUDA tensor (the
+    read-bandwidth diagnostic); sink is a CUDA int32 tensor of >= 1 element."""
+    if not (buf.is_cuda and buf.is_contiguous()):
+        raise ValueError("buf: must be a contiguous CUDA tensor")
+    sp = _ptr(sink, torch.int32, "sink")
+    _check(lib().md_stream_read(buf.data_ptr(), buf.numel() * buf.element_size(), sp, _stream(stream)),
+           "md_stream_read")
 
 
 def version() -> int:
