@@ -53,8 +53,8 @@ def heads_bytes(w):
     return w.head_weight_bytes() + 2 * w.M * w.d + 8 * w.M * w.K * w.kmax + extra
 
 
-TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
-                               "heads_traffic_prof-8b-v32000.md")
+PROFILE_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
+TRAFFIC_PROFILE = os.path.join(PROFILE_DIR, "heads_traffic_prof-8b-v32000.md")
 HEADS_SOURCES = ("heads.cuh", "common.cuh")
 
 
@@ -94,24 +94,38 @@ def heads_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_heads_traffic(w):
-    """DRAM bytes of one streaming heads call: the ratio DRAM traffic /
-    algorithmic bytes recorded from an ncu capture (profiles/
-    heads_traffic_prof-8b-v32000.md) times this workload's algorithmic bytes.
-    None off the one-row streaming path that was captured, or when the heads
-    sources changed since the capture (digest mismatch)."""
-    if w.M > 1 or not os.path.exists(TRAFFIC_PROFILE):
+def _traffic_record(path):
+    """(bytes per call, ratio to the algorithmic bytes, digest) from a traffic
+    profile, or None."""
+    if not os.path.exists(path):
         return None
-    ratio = digest = None
-    with open(TRAFFIC_PROFILE) as fh:
+    rec = {}
+    with open(path) as fh:
         for line in fh:
-            if line.startswith("traffic_per_algorithmic_byte:"):
-                ratio = float(line.split(":")[1])
-            elif line.startswith("heads_source_digest:"):
-                digest = line.split(":")[1].split()[0]
-    if ratio is None or digest != heads_source_digest():
-        return None
-    return ratio * heads_bytes(w)
+            for key in ("traffic_per_call_bytes", "traffic_per_algorithmic_byte", "heads_source_digest"):
+                if line.startswith(key + ":"):
+                    rec[key] = line.split(":")[1].split()[0]
+    return rec
+
+
+def measured_heads_traffic(w):
+    """DRAM bytes of one one-row streaming heads call, from ncu captures
+    recorded under profiles/: the capture of this very workload when there is
+    one (the 70B call, whose metrics take a single ncu pass), else the ratio
+    DRAM traffic / algorithmic bytes of the 8B-shaped V 32000 capture times this
+    workload's algorithmic bytes. Returns (bytes, source) or (None, None) off the
+    captured path or when the heads sources changed since the capture."""
+    if w.M > 1:
+        return None, None
+    digest = heads_source_digest()
+    own = _traffic_record(os.path.join(PROFILE_DIR, f"heads_traffic_{w.name}.md"))
+    if own and own.get("heads_source_digest") == digest and "traffic_per_call_bytes" in own:
+        return float(own["traffic_per_call_bytes"]), f"profiles/heads_traffic_{w.name}.md (this workload)"
+    rec = _traffic_record(TRAFFIC_PROFILE)
+    if rec and rec.get("heads_source_digest") == digest and "traffic_per_algorithmic_byte" in rec:
+        return (float(rec["traffic_per_algorithmic_byte"]) * heads_bytes(w),
+                "profiles/heads_traffic_prof-8b-v32000.md scaled by algorithmic bytes")
+    return None, None
 
 
 def slowest_rank_ms(ms: float, world: int, device=None) -> float:
@@ -584,10 +598,10 @@ def run_medusa(args, w):
             roof["frac_nominal"] = roof["achieved"] / NOMINAL_HBM_GBS
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["above_peak"] = roof["frac"] > 1.0
-        roof["traffic"] = args.traffic if args.traffic is not None else measured_heads_traffic(w)
-        roof["traffic_source"] = ("--traffic" if args.traffic is not None else
-                                  "profiles/heads_traffic_prof-8b-v32000.md scaled by algorithmic bytes"
-                                  if roof["traffic"] is not None else None)
+        if args.traffic is not None:
+            roof["traffic"], roof["traffic_source"] = args.traffic, "--traffic"
+        else:
+            roof["traffic"], roof["traffic_source"] = measured_heads_traffic(w)
         roof["avg_ms"] = heads_ms
         roof["peak_source"] = peaks["source"]
         ab = attention_bytes(w, P)
