@@ -55,7 +55,7 @@ def heads_bytes(w):
 
 PROFILE_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
 TRAFFIC_PROFILE = os.path.join(PROFILE_DIR, "heads_traffic_prof-8b-v32000.md")
-HEADS_SOURCES = ("heads.cuh", "common.cuh")
+HEADS_SOURCES = ("heads.cuh", "heads_skinny.cuh", "heads_gemm.cuh", "heads_gemm2.cuh", "common.cuh")
 
 
 def hydra_levels(parent):
@@ -109,18 +109,19 @@ def _traffic_record(path):
 
 
 def measured_heads_traffic(w):
-    """DRAM bytes of one one-row streaming heads call, from ncu captures
-    recorded under profiles/: the capture of this very workload when there is
-    one (the 70B call, whose metrics take a single ncu pass), else the ratio
-    DRAM traffic / algorithmic bytes of the 8B-shaped V 32000 capture times this
-    workload's algorithmic bytes. Returns (bytes, source) or (None, None) off the
-    captured path or when the heads sources changed since the capture."""
-    if w.M > 1:
-        return None, None
+    """DRAM bytes of one heads call, from ncu captures recorded under
+    profiles/: the capture of this very workload when there is one (its
+    metrics take a single ncu pass, so full-size calls are captured directly),
+    else, for one-row streaming calls, the ratio DRAM traffic / algorithmic
+    bytes of the 8B-shaped V 32000 capture times this workload's algorithmic
+    bytes. Returns (bytes, source), or (None, None) when there is no capture
+    or the heads sources changed since it was taken."""
     digest = heads_source_digest()
     own = _traffic_record(os.path.join(PROFILE_DIR, f"heads_traffic_{w.name}.md"))
     if own and own.get("heads_source_digest") == digest and "traffic_per_call_bytes" in own:
         return float(own["traffic_per_call_bytes"]), f"profiles/heads_traffic_{w.name}.md (this workload)"
+    if w.M > 1:
+        return None, None
     rec = _traffic_record(TRAFFIC_PROFILE)
     if rec and rec.get("heads_source_digest") == digest and "traffic_per_algorithmic_byte" in rec:
         return (float(rec["traffic_per_algorithmic_byte"]) * heads_bytes(w),
