@@ -120,7 +120,9 @@ def _clear(decisions):
 
 @pytest.mark.parametrize("kph,n,B,V,tau,tau_q", [((4, 3, 2, 2), 16, 32, 1024, 0.7, 0.7),
                                                   ((10, 10, 10, 10), 64, 16, 128256, 0.7, 1.0),
-                                                  ((1, 1, 1, 1), 4, 16, 32000, 1.0, 0.8)])
+                                                  ((1, 1, 1, 1), 4, 16, 32000, 1.0, 0.8),
+                                                  # a vocabulary that splits unevenly over the 8 CTAs
+                                                  ((4, 3, 2, 2), 16, 24, 1030, 0.9, 0.7)])
 def test_rejection_acceptance_matches_oracle(kph, n, B, V, tau, tau_q):
     case = _case(n + B, kph, n, B, V, B + 3, 0.6, tau, tau_q)
     parent, rank, tokens, tl, hl, head_row, ua, ur = case
