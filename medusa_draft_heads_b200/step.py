@@ -39,9 +39,12 @@ class MedusaStep:
         self.anc = torch.empty((self.T, (self.T + 31) // 32), **i32)
         self.pos = torch.empty((B, self.T), **i32)
         self.attn_out = torch.empty((B, self.T, Hq, dh), **f32)
-        self.accept_len = torch.empty((B,), **i32)
-        self.path = torch.empty((B, K + 1), **i32)
-        self.bonus = torch.empty((B,), **i32)
+        # the step's result in one buffer (accept_len [B], path [B, K+1],
+        # bonus [B]), so a caller reads it back with one copy
+        self.result = torch.empty((B * (K + 3),), **i32)
+        self.accept_len = self.result[:B]
+        self.path = self.result[B:B * (K + 2)].view(B, K + 1)
+        self.bonus = self.result[B * (K + 2):]
         self.new_prefix_len = torch.empty((B,), **i32)
         self.next_root = torch.empty((B,), **i32)
         self.next_head_row = torch.empty((B,), **i32)
