@@ -866,13 +866,6 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
     copied = torch.cuda.Event()
 
     def e2e_step():
-        # the heads' inputs and the heads first: they are the critical path
-        h.copy_(host["h"], non_blocking=True)
-        if "u_draft" in host:          # the draws' uniforms feed the heads
-            step.u_draft.copy_(host["u_draft"], non_blocking=True)
-        root.copy_(host["root"], non_blocking=True)
-        prefix.copy_(host["prefix"], non_blocking=True)
-        step.heads(h, W1, b1, Wv)
         with torch.cuda.stream(copy_stream):
             q0.copy_(host["q"], non_blocking=True)
             for b in range(w.B):
@@ -883,6 +876,12 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
                 if name in host:
                     getattr(step, name).copy_(host[name], non_blocking=True)
             copied.record(copy_stream)
+        h.copy_(host["h"], non_blocking=True)
+        if "u_draft" in host:          # the draws' uniforms feed the heads
+            step.u_draft.copy_(host["u_draft"], non_blocking=True)
+        root.copy_(host["root"], non_blocking=True)
+        prefix.copy_(host["prefix"], non_blocking=True)
+        step.heads(h, W1, b1, Wv)
         step.build(root, prefix, head_row)
         stream.wait_event(copied)
         step.attention(q0, kc0, vc0, prefix)
@@ -908,8 +907,8 @@ def run_e2e(args, w, step, h, W1, b1, Wv, root, prefix, head_row, sets, stream, 
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "per step: h, root token, prefix lengths, q, the tree tokens' K/V and the target logits "
                     "copied in from pinned host memory (q, K/V and logits on a second stream, overlapping the "
-                    "heads, which are enqueued first); accept_len, path and bonus copied out in one copy; both "
-                    "streams synchronised after every step"}
+                    "heads); accept_len, path and bonus copied out in one copy; both streams synchronised after "
+                    "every step"}
 
 
 def cpu_baseline(w, args):
