@@ -75,8 +75,10 @@ enum {
 
 /* Supported ranges (anything else: MD_ERR_UNSUPPORTED).
  *   heads:     1 <= K <= 8, 1 <= k_i <= kmax <= 16, d % 64 == 0, V % 8 == 0,
- *              V >= 256, 1 <= M <= 4096 (M <= 4: CUDA-core weight stream;
- *              M > 4: tcgen05 tensor-core GEMM, h and b1 16-byte aligned).
+ *              V >= 256, 1 <= M <= 4096 (M = 1: CUDA-core weight stream;
+ *              2 <= M <= 64: tcgen05 weight stream with the weights as the
+ *              MMA's M; M > 64: tcgen05 GEMM on 128-row tiles; from two rows
+ *              h and b1 must be 16-byte aligned).
  *   tree:      1 <= T <= 128, depth <= K.
  *   attention: dh in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16.
  */
@@ -220,7 +222,7 @@ MD_API md_status md_medusa_heads_sampled(const md_bf16* h, const md_bf16* W1, co
  *   array are rejected with MD_ERR_WORKSPACE before anything is launched. The
  *   scratch of the tensor-core path grows with the device's SM count, so the
  *   largest admitted M depends on the GPU: on a 148-SM B200 at d = 8192,
- *   V = 128256, K = 4, kmax = 10 it is M = 74. Callers that need a guarantee
+ *   V = 128256, K = 4, kmax = 10 every M up to 433 fits. Callers that need a guarantee
  *   compare md_heads_workspace(...) with MD_HEADS_STATIC_SCRATCH_BYTES on
  *   their device.
  * - The first call on each device looks up the array's device address

@@ -27,7 +27,8 @@ constexpr int kZPad = 8;            // z row i is stored as 8 bf16 (one per m), 
 constexpr int kW1Threads = 256;
 constexpr int kW1TileO = 256;       // phase-1 output columns per CTA
 constexpr int kW1MaxRows = 2048;    // phase-1 hidden rows per CTA (split-K)
-constexpr int kMaxM = 4;        // rows beyond this take the tensor-core path (faster from M = 5 on)
+constexpr int kMaxM = 4;        // rows these kernels support; the launchers use them for one row (the
+                                // tensor-core weight stream is faster from two)
 constexpr uint32_t kStageWBytes = kStageRows * kTileV * 2;  // 32 KB
 constexpr uint32_t kStageZBytes = kStageRows * kZPad * 2;   // 1 KB
 constexpr int kSmemBudget = 227 * 1024;
