@@ -55,7 +55,14 @@ def heads_bytes(w):
 
 PROFILE_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
 TRAFFIC_PROFILE = os.path.join(PROFILE_DIR, "heads_traffic_prof-8b-v32000.md")
-HEADS_SOURCES = ("heads.cuh", "heads_skinny.cuh", "heads_gemm.cuh", "heads_gemm2.cuh", "common.cuh")
+# The kernel sources each heads path runs (a traffic capture is tied to them).
+HEADS_SOURCES = {"stream": ("heads.cuh", "common.cuh"),
+                 "weights-as-m": ("heads.cuh", "heads_skinny.cuh", "common.cuh"),
+                 "row-tiles": ("heads.cuh", "heads_gemm.cuh", "heads_gemm2.cuh", "common.cuh")}
+
+
+def heads_path(M: int) -> str:
+    return "stream" if M == 1 else "weights-as-m" if M <= 64 else "row-tiles"
 
 
 def hydra_levels(parent):
@@ -78,14 +85,14 @@ def hydra_flops(w, levels):
     return sum(2 * w.B * n * (w.d * w.d + w.d * w.V) for n in levels)
 
 
-def heads_source_digest() -> str:
+def heads_source_digest(path: str = "stream") -> str:
     """sha256 (first 16 hex digits) of the heads sources with comments and
     whitespace removed: a change of code invalidates a recorded capture, a
     change of wording does not."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in HEADS_SOURCES:
+    for f in HEADS_SOURCES[path]:
         with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "medusa_draft_heads_b200", "csrc", f)) as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -116,7 +123,7 @@ def measured_heads_traffic(w):
     bytes of the 8B-shaped V 32000 capture times this workload's algorithmic
     bytes. Returns (bytes, source), or (None, None) when there is no capture
     or the heads sources changed since it was taken."""
-    digest = heads_source_digest()
+    digest = heads_source_digest(heads_path(w.M))
     own = _traffic_record(os.path.join(PROFILE_DIR, f"heads_traffic_{w.name}.md"))
     if own and own.get("heads_source_digest") == digest and "traffic_per_call_bytes" in own:
         return float(own["traffic_per_call_bytes"]), f"profiles/heads_traffic_{w.name}.md (this workload)"
