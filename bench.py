@@ -204,6 +204,20 @@ def read_stream_gbs(dev, nbytes=1 << 32, reps=10):
     return nbytes / (ms / 1000.0) / 1e9
 
 
+def attention_launches(w) -> int:
+    """The tcgen05 tree attention is one kernel (its KV splits merge through
+    distributed shared memory); GQA groups that do not divide 128 rows take
+    the CUDA-core kernel and its merge kernel."""
+    return 1 if 128 % (w.Hq // w.Hkv) == 0 else 2
+
+
+def step_launches(w) -> int:
+    """This library's kernels in one step: heads 3 (residual block, projection
+    with the top-k, merge), tree build 1, attention, acceptance 2 (row scan or
+    per-row draw, then the walk; 1 for the rejection rule)."""
+    return 3 + 1 + attention_launches(w) + (1 if w.mode == "rejection" else 2)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -635,8 +649,7 @@ def run_medusa(args, w):
             "attention": {"bytes": ab, "flops": af, "gbs": ab / (attn_ms / 1000) / 1e9,
                           "tflops": af / (attn_ms / 1000) / 1e12},
             "accept": {"bytes": accept_bytes(w), "gbs": accept_bytes(w) / (acc_ms / 1000) / 1e9},
-            # heads 3, tree build 1, attention 2 (main + merge, or chunks + merge), acceptance 2 (1 rejection)
-            "gpu_launches": (3 + 1 + 2 + (1 if w.mode == "rejection" else 2)) * args.steps,
+            "gpu_launches": step_launches(w) * args.steps,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -696,7 +709,7 @@ def run_part(args, w):
                  sdev.fill_normal(torch.empty((w.B, w.Hkv, w.S_max, w.dh), **bf), seed + i, "v_cache", 1.0))
                 for i in range(nsets)]
         call = lambda i: step.attention(*sets[i % nsets], prefix)                # noqa: E731
-        nbytes, nflops, launches = attention_bytes(w, P), attention_flops(w, P), 2
+        nbytes, nflops, launches = attention_bytes(w, P), attention_flops(w, P), attention_launches(w)
     elif args.part == "commit":
         tokens = synth.synthetic_tree_tokens(seed, w.B, np.array(step.tree.parent), w.V)
         logits = synth.planted_logits_device(seed, np.array(step.tree.parent), tokens, w.V, w.accept,
