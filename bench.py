@@ -62,7 +62,7 @@ HEADS_SOURCES = {"stream": ("heads.cuh", "common.cuh"),
 
 
 def heads_path(M: int) -> str:
-    return "stream" if M == 1 else "weights-as-m" if M <= 64 else "row-tiles"
+    return "stream" if M == 1 else "weights-as-m" if M <= 32 else "row-tiles"
 
 
 def hydra_levels(parent):
@@ -601,7 +601,7 @@ def run_medusa(args, w):
         hb = heads_bytes(w)
         hf = heads_flops(w)
         heads_ms = float(per_call[:, 0].mean())
-        if w.M > 64:     # row-tile tensor-core GEMMs: bound by the bf16 tensor pipe
+        if w.M > 32:     # row-tile tensor-core GEMMs: bound by the bf16 tensor pipe
             roof = {"kernel": "md_medusa_heads (tcgen05 GEMMs: residual block, vocabulary projection + top-k; merge)",
                     "bound": "tensor", "achieved": hf / (heads_ms / 1000.0) / 1e12,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
@@ -843,7 +843,7 @@ def run_sweep(args):
                     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
                     tot = float(np.mean([e[0].elapsed_time(e[4]) for e in evs]))
                     print(json.dumps({"sweep": w.name, "B": B, "tree": tree, "prefix": P, "mode": mode,
-                                      "heads_path": ("tcgen05-pair-gemm" if w.M > 128 else "tcgen05-gemm" if w.M > 64
+                                      "heads_path": ("tcgen05-pair-gemm" if w.M > 128 else "tcgen05-gemm" if w.M > 32
                                                      else "tcgen05-weights-as-m" if w.M > 1 else "cuda-core-stream"),
                                       "steps_per_s": 1000.0 / tot, "ms_per_step": tot,
                                       "ms": {"heads": float(per[:, 0].mean()), "build": float(per[:, 1].mean()),

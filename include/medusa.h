@@ -76,8 +76,8 @@ enum {
 /* Supported ranges (anything else: MD_ERR_UNSUPPORTED).
  *   heads:     1 <= K <= 8, 1 <= k_i <= kmax <= 16, d % 64 == 0, V % 8 == 0,
  *              V >= 256, 1 <= M <= 4096 (M = 1: CUDA-core weight stream;
- *              2 <= M <= 64: tcgen05 weight stream with the weights as the
- *              MMA's M; M > 64: tcgen05 GEMM on 128-row tiles; from two rows
+ *              2 <= M <= 32: tcgen05 weight stream with the weights as the
+ *              MMA's M; M > 32: tcgen05 GEMM on 128-row tiles; from two rows
  *              h and b1 must be 16-byte aligned).
  *   tree:      1 <= T <= 128, depth <= K.
  *   attention: dh in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16.

@@ -1,4 +1,4 @@
-// Medusa draft heads on the tensor cores for a few hidden rows (2 .. 64),
+// Medusa draft heads on the tensor cores for a few hidden rows (2 .. 32),
 // with the weights on the MMA's M side.
 //
 // Source: "Medusa heads versus separate draft model", sections "What each one
@@ -12,7 +12,7 @@
 // from two rows on, and a 128-row MMA tile pads M to 128. Here
 // the product is computed transposed, D^T = W^T x^T: 128 output columns of the
 // weights form the MMA's M (the weight tile is N-major as TMA brings it from
-// the input-major matrix) and the rows form its N (NR = 16, 32 or 64, rows
+// the input-major matrix) and the rows form its N (NR = 16 or 32, rows
 // K-major). A 64-deep stage moves 32 KB of weights plus NR x 128 B of rows and
 // costs 8 MMAs of 128 x NR x 16, well below the time of its bytes.
 //
@@ -45,7 +45,7 @@ constexpr uint32_t kWBox = 64 * kBK * 2;     // 8 KB: 64 reduction rows x 64 col
 constexpr uint32_t kWBytes = 4 * kWBox;      // 32 KB per stage
 constexpr int kThreads = 192;
 constexpr int kChunk = 16;                   // rows per tcgen05.ld in the epilogue
-constexpr int kMinRows = 2, kMaxRows = 64;   // the launcher's range of rows for this path
+constexpr int kMinRows = 2, kMaxRows = 32;   // the launcher's range of rows for this path
 
 enum { EPI_SILU = 0, EPI_TOPK = 1 };
 

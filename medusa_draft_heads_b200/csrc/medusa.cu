@@ -359,11 +359,11 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
 }
 
-// ---------------- tensor-core heads with the weights as M (5 .. 64 rows) ----------------
+// ---------------- tensor-core heads with the weights as M (2 .. 32 rows) ----------------
 // Workspace: z [K, NR, d] bf16, two partial-sum slots per CTA, one ticket per
 // unit of both phases, and the phase-2 candidates [M, K, G2, kmax].
 struct SkinnyPlan {
-  int NR;                  // rows padded to 16, 32 or 64 (the MMA's N)
+  int NR;                  // rows padded to 16 or 32 (the MMA's N)
   int S, nt1, nt2;         // stages per unit, column tiles of phase 1 (d) and phase 2 (V)
   int G1, G2;              // CTAs of the two phases
   size_t off_z, off_part, off_tick, off_cval, off_cid, bytes;
@@ -372,13 +372,15 @@ struct SkinnyPlan {
 inline bool skinny_rows(int M) { return M >= md::skinny::kMinRows && M <= md::skinny::kMaxRows; }
 
 // The CUDA-core stream serves one row; from two rows the tensor cores (its
-// FMA work grows with M: 1.50 vs 1.32 ms at two rows of 70B heads).
+// FMA work grows with M: 1.50 vs 1.32 ms at two rows of 70B heads); from 33
+// rows the 128-row GEMM tiles (1.44 ms at 65 rows against 1.48 ms for the
+// weights-as-M kernel at 64: N = 64 leaves four stages and a heavier epilogue).
 inline bool stream_rows(int M) { return M < md::skinny::kMinRows; }
 
 SkinnyPlan skinny_plan(int M, int d, int V, int K, int kmax) {
   using md::heads::align256;
   SkinnyPlan p;
-  p.NR = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.NR = M <= 16 ? 16 : 32;
   p.S = d / md::skinny::kBK;
   p.nt1 = (d + md::skinny::kTile - 1) / md::skinny::kTile;
   p.nt2 = (V + md::skinny::kTile - 1) / md::skinny::kTile;
@@ -464,7 +466,7 @@ md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, 
 
 struct SharedPlan {
   bool stream;                 // M*K == 1: CUDA-core weight stream
-  bool skinny;                 // 2 <= M*K <= 64: tensor cores with the weights as M; else row-tile GEMMs
+  bool skinny;                 // 2 <= M*K <= 32: tensor cores with the weights as M; else row-tile GEMMs
   md::heads::Plan p1, p2;      // streaming: phase-1 plan (M rows, K heads), phase-2 plan (M*K rows, 1 head)
   GemmPlan g1, g2;             // tensor cores: phase 1 (M rows, K heads), phase 2 (M*K rows, 1 head)
   size_t off2, bytes;
@@ -474,7 +476,7 @@ struct SharedPlan {
   size_t off_z, off_part, off_tick, off_cval, off_cid;
 };
 
-inline int skinny_pad(int rows) { return rows <= 16 ? 16 : (rows <= 32 ? 32 : 64); }
+inline int skinny_pad(int rows) { return rows <= 16 ? 16 : 32; }
 
 SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
   using md::heads::align256;
@@ -871,7 +873,7 @@ void heads_zero_range(int M, int d, int V, int K, int kmax, size_t* off, size_t*
 }
 
 // md_medusa_heads and md_medusa_heads_sampled: checks, then the streaming
-// (one row), weights-as-M (2 .. 64 rows) or row-tile tensor-core path.
+// (one row), weights-as-M (2 .. 32 rows) or row-tile tensor-core path.
 // gumbel_u null: top-k of the logits; else the top-k of the Gumbel keys
 // logit * inv_tau - ln(-ln u). zeroed: heads_zero_range is already zero.
 md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, int32_t M,
@@ -896,10 +898,7 @@ md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, con
     if (pl.NR == 16)
       return launch_heads_skinny<16>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
                                      logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
-    if (pl.NR == 32)
-      return launch_heads_skinny<32>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
-                                     logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
-    return launch_heads_skinny<64>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
+    return launch_heads_skinny<32>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
                                    logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
   }
   if (!stream_rows(M)) {
@@ -1074,10 +1073,7 @@ md_status md_medusa_heads_shared(const md_bf16* h, const md_bf16* W1, const md_b
                                             logits_dbg, w, st);
     MD_SHARED_SKINNY(16, 16)
     MD_SHARED_SKINNY(16, 32)
-    MD_SHARED_SKINNY(16, 64)
     MD_SHARED_SKINNY(32, 32)
-    MD_SHARED_SKINNY(32, 64)
-    MD_SHARED_SKINNY(64, 64)
 #undef MD_SHARED_SKINNY
     return MD_ERR_UNSUPPORTED;
   }

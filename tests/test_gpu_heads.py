@@ -96,7 +96,7 @@ def test_heads_reject_bad_arguments():
                         vals, ws)
 
 
-# ------------- tensor-core paths (M > 1: weights as M up to 64 rows, row tiles up to 128, CTA pairs beyond) -------------
+# ------------- tensor-core paths (M > 1: weights as M up to 32 rows, row tiles up to 128, CTA pairs beyond) -------------
 
 @pytest.mark.parametrize("M,d,V,kph", [(9, 256, 1024, (4, 3, 2, 2)), (40, 320, 1000, (10, 10, 10, 10)),
                                        (130, 512, 2056, (16, 1, 7, 3)), (520, 256, 4096, (10, 10, 10, 10))])
@@ -131,15 +131,16 @@ def test_tensor_core_fused_equals_debug_run():
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
-# ------------- tensor cores with the weights as the MMA's M (5 .. 64 rows) -------------
+# ------------- tensor cores with the weights as the MMA's M (2 .. 32 rows) -------------
 
 @pytest.mark.parametrize("M,d,V,kph", [
+    (2, 512, 2056, (10, 10, 10, 10)),        # the smallest row count of this path
     (5, 1024, 8192, (10,)),                  # one head: 4 phase-1 units over 64 CTAs, 16 parts each
     (10, 4096, 4096, (10,)),                 # a Hydra level's row count; units cut into many parts
     (16, 576, 3000, (4, 3, 2, 2)),           # 9 stages per unit, ragged last vocabulary tile
-    (33, 512, 1000, (10, 10, 10, 10)),       # 64-row padding, 33 live rows
-    (64, 256, 2056, (16, 1, 7, 3)),          # the largest row count of this path
-    (100, 256, 1024, (10, 10, 10, 10)),      # 65 .. 128 rows: one 128-row tile per CTA
+    (17, 512, 1000, (10, 10, 10, 10)),       # 32-row padding, 17 live rows
+    (32, 256, 2056, (16, 1, 7, 3)),          # the largest row count of this path
+    (33, 256, 1024, (10, 10, 10, 10)),       # 33 .. 128 rows: one 128-row tile per CTA
 ])
 def test_weights_as_m_heads_match_oracle(M, d, V, kph):
     h, W1, b1, Wv = head_weights(500 + M, d, V, len(kph), M)
@@ -177,7 +178,8 @@ def _run_shared(h, W1, b1, Wv, kph, kmax=None):
 @pytest.mark.parametrize("M,d,V,kph", [(1, 256, 1024, (10,)),                      # one row: streaming
                                        (1, 256, 1024, (4, 3, 2, 2)), (1, 512, 2056, (10, 10, 10, 10)),
                                        (2, 320, 1000, (16, 1)), (3, 256, 4096, (10, 10, 10, 10)),
-                                       (12, 576, 3000, (16, 7, 3, 1)),             # 48 rows after 12-row phase 1
+                                       (6, 576, 3000, (16, 7, 3, 1)),              # 24 rows after a 6-row phase 1
+                                       (12, 576, 3000, (16, 7, 3, 1)),             # 48 rows: row-tile GEMMs
                                        (130, 256, 1024, (7, 3, 2))])
 def test_shared_projection_matches_oracle(M, d, V, kph):
     K = len(kph)
