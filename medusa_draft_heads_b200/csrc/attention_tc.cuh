@@ -9,15 +9,16 @@
 // CTA = (KV split, 128-row query tile, KV head, request); the grid is sized to
 // one wave. The 128 query rows are (tree token, query head of the group) pairs,
 // loaded by one 3-D TMA box straight out of q[B, T, Hq, dh]. The CTA walks its
-// share of 128-key chunks:
+// share of CH-key chunks (CH = 64 or 128, see Cfg):
 //
-//   warp 0     TMA: the Q tile once, then K and V chunks into two 3-deep rings
+//   warp 0     TMA: the Q tile once, then K and V chunks into two rings
 //              (a K slot frees when its S is done, a V slot when its P V is)
-//   warp 1     one thread issues S_c = Q K_c^T into TMEM (three buffers, three
-//              chunks ahead) and O += P_c V_c into one TMEM accumulator that
-//              lives across chunks, with P_c read from TMEM
-//   warps 2-9  two warps per TMEM lane quarter, each taking half of the keys of
-//              a row (row maxima are exchanged through shared memory): read
+//   warp 1     one thread issues S_c = Q K_c^T into TMEM (one buffer per ring
+//              slot, that many chunks ahead) and O += P_c V_c into one TMEM
+//              accumulator that lives across chunks, with P_c read from TMEM
+//   softmax    one warp per TMEM lane quarter and 64 keys of the chunk (two per
+//              quarter for 128-key chunks; row maxima are then exchanged
+//              through shared memory): read
 //              S_c from TMEM, apply the scale and -- only in chunks that reach
 //              the tree slots -- the tree mask (a key at slot >= P_b is tree
 //              node slot - P_b, visible iff it is an ancestor-or-self), then
@@ -28,9 +29,9 @@
 //              than 2^8; O and the row sum are then rescaled in place.
 //
 // Because P_c lives in S_c's buffer, the softmax of chunk c + 1 never waits for
-// P_c V_c (only a rescale of O does), and with three buffers S_{c+1}, S_{c+2}
-// are computed while the softmax works on c: the softmax warps and the tensor
-// pipe work on different chunks at the same time.
+// P_c V_c (only a rescale of O does), and the next buffers' S are computed
+// while the softmax works on c: the softmax warps and the tensor pipe work on
+// different chunks at the same time.
 //
 // The KV splits of one (request, KV head, row tile) are the CTAs of one
 // cluster. Each stages its split's unnormalised O and per-row (m, sum) in its
@@ -46,26 +47,36 @@ namespace md {
 namespace attn_tc {
 
 constexpr int kBM = 128;        // query rows per CTA
-constexpr int kBN = 128;        // keys per chunk
-constexpr int kSoftWarps = 8;
-constexpr int kThreads = 64 + kSoftWarps * 32;
-constexpr uint32_t kTmemCols = 512;
+constexpr int kKeysPerWarp = 64;   // keys of a chunk one softmax warp takes for its 32 rows
 constexpr float kRescaleLog2 = 8.0f;   // lazy rescale threshold (factor 256)
 constexpr int kMaxSplits = 8;    // KV splits of one tile = CTAs of one cluster (portable size)
 
-constexpr int kStages = 3;      // K / V ring depth
-constexpr int kSBufs = 3;       // S / P buffers in TMEM (3 x 128 columns + O)
-
-template <int DH>
+// Two shapes of the same pipeline. CH = 128: 128-key chunks, two softmax warps
+// per TMEM lane quarter (64 keys each, row maxima exchanged), three S/P buffers
+// and a 3-deep K/V ring, all 512 TMEM columns: one CTA per SM. CH = 64: 64-key
+// chunks, one softmax warp per lane quarter, two S/P buffers, a 2-deep ring and
+// 256 TMEM columns, small enough for two CTAs per SM, so that one CTA's
+// prologue and split merge overlap the other's chunk loop.
+template <int DH, int CH>
 struct Cfg {
+  static constexpr int kBN = CH;                              // keys per chunk
+  static constexpr int kWPQ = CH / kKeysPerWarp;              // softmax warps per TMEM lane quarter
+  static constexpr int kSoftWarps = 4 * kWPQ;
+  static constexpr int kThreads = 64 + kSoftWarps * 32;
+  static constexpr int kStages = CH == 128 ? 3 : 2;           // K / V ring depth
+  static constexpr int kSBufs = CH == 128 ? 3 : 2;            // S / P buffers in TMEM (+ O)
+  static constexpr uint32_t kTmemCols = CH == 128 ? 512 : 256;
+  static constexpr int kMinBlocks = CH == 128 ? 1 : 2;        // resident CTAs per SM
   static constexpr int KB = DH / 64;                          // 64-element blocks of the head dim
   static constexpr uint32_t kQBytes = KB * kBM * 128;         // Q tile, K-major SW128
   static constexpr uint32_t kKBytes = KB * kBN * 128;         // K chunk, K-major SW128
   static constexpr uint32_t kVBytes = KB * kBN * 128;         // V chunk, N(dh)-major SW128
   static constexpr uint32_t kStage = kKBytes + kVBytes;
   static constexpr int kSmem = kQBytes + kStages * kStage + 1024 + 256 + 1024;  // + barriers, maxima
-  // the epilogue stages O, the merge weights and (m, l) over the idle K/V ring
-  static_assert(kBM * (DH + 4) * 4 + kBM * (kMaxSplits + 1) * 4 + kBM * 8 <= kStages * kStage, "staging");
+  // the epilogue stages O, the merge weights and (m, l) over the idle Q tile and K/V ring
+  static_assert(kBM * (DH + 4) * 4 + kBM * (kMaxSplits + 1) * 4 + kBM * 8 <= kQBytes + kStages * kStage,
+                "staging");
+  static_assert(kSBufs * kBN + DH <= int(kTmemCols), "TMEM");
 };
 
 struct Args {
@@ -97,11 +108,13 @@ __device__ __forceinline__ uint64_t visible_bits(uint64_t lo, uint64_t hi, int n
   return hi >> (n0 - 64);
 }
 
-template <int DH>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int DH, int CH>
+__global__ void __launch_bounds__(Cfg<DH, CH>::kThreads, Cfg<DH, CH>::kMinBlocks)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ TreeParams tp, Args a) {
-  using C = Cfg<DH>;
+  using C = Cfg<DH, CH>;
+  constexpr int kBN = C::kBN, kStages = C::kStages, kSBufs = C::kSBufs, kSoftWarps = C::kSoftWarps;
+  constexpr uint32_t kTmemCols = C::kTmemCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;
@@ -182,10 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tO = tmem + kSBufs * kBN;  // O at columns [384, 384 + DH)
   const int kvrow = b * a.Hkv + hk;
   const int tpt = kBM / a.G;                // tree tokens per query tile
-  // epilogue staging over the K/V ring: O [128][kLd] (padded rows: conflict-free
+  // epilogue staging over the Q tile and the K/V ring: O [128][kLd] (padded rows: conflict-free
   // 16-byte accesses), merge weights [128][kMaxSplits + 1] (1/L last), (m, l) [128]
   constexpr int kLd = DH + 4;
-  float* sO = reinterpret_cast<float*>(sKV);
+  float* sO = reinterpret_cast<float*>(smem);   // over the Q tile and the K/V ring
   float* sW = sO + kBM * kLd;
   float2* sML = reinterpret_cast<float2*>(sW + kBM * (kMaxSplits + 1));
 
@@ -294,9 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------- softmax rows -------------------------------
-    const int sw = warp - 2;                     // 0..7
+    const int sw = warp - 2;                     // 0 .. kSoftWarps-1
     const int q = warp & 3;                      // TMEM lane quarter
-    const int half = sw >> 2;                    // which 64 keys of the chunk (and of O's columns)
+    const int half = sw >> 2;                    // which 64 keys of the chunk (and which part of O's
+                                                 // columns); 0 when one warp takes the whole chunk
     const int r = q * 32 + lane;                 // row of the tile = TMEM lane
     const int grow = rt * kBM + r;               // row within (request, KV head)
     const bool live = grow < a.R;
@@ -305,7 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t anc_lo = (uint64_t(tp.anc[t][1]) << 32) | tp.anc[t][0];
     const uint64_t anc_hi = (uint64_t(tp.anc[t][3]) << 32) | tp.anc[t][2];
     const float sc = a.scale_log2;
-    constexpr int kHalf = kBN / 2;
+    constexpr int kHalf = kKeysPerWarp;
+    constexpr int kOCols = DH / C::kWPQ;         // O columns this warp rescales and stages
     float run_m = -INFINITY, run_l = 0.f;
     bool ok = true;
     // Every iteration runs both named barriers, so a wait that gives up (ok =
@@ -337,13 +352,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[j + i]);
         mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
-      // exchange the half maxima with the partner warp (same lane quarter); after
-      // the first barrier both warps have read their S columns, so either may
-      // overwrite the buffer with P
-      xmax[half * kBM + r] = mx;
-      named_bar_sync(1 + q, 64);
-      mx = fmaxf(mx, xmax[(half ^ 1) * kBM + r]);
-      named_bar_sync(1 + q, 64);                 // both have read before the slots are reused
+      if constexpr (C::kWPQ == 2) {
+        // exchange the half maxima with the partner warp (same lane quarter);
+        // after the first barrier both warps have read their S columns, so
+        // either may overwrite the buffer with P
+        xmax[half * kBM + r] = mx;
+        named_bar_sync(1 + q, 64);
+        mx = fmaxf(mx, xmax[(half ^ 1) * kBM + r]);
+        named_bar_sync(1 + q, 64);               // both have read before the slots are reused
+      }
       mx = (mx == -INFINITY) ? -INFINITY : mx * sc;
       if (!ok) continue;
       const bool grow_m = mx > run_m + kRescaleLog2 || (run_m == -INFINITY && mx != -INFINITY);
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int e0 = half * (DH / 2); e0 < (half + 1) * (DH / 2); e0 += 32) {
+        for (int e0 = half * kOCols; e0 < (half + 1) * kOCols; e0 += 32) {
           float o[32];
           tmem_ld32(tO + lane_off + e0, o);
 #pragma unroll
@@ -405,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__all_sync(0xffffffffu, mbar_wait(smem_u32(o_last), 0))) {
         tc_fence_after();
 #pragma unroll
-        for (int e0 = half * (DH / 2); e0 < (half + 1) * (DH / 2); e0 += 32) {
+        for (int e0 = half * kOCols; e0 < (half + 1) * kOCols; e0 += 32) {
           float o[32];
           tmem_ld32(tO + lane_off + e0, o);
 #pragma unroll
@@ -417,9 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok) set_status(MD_DEV_TIMEOUT);
-    xmax[half * kBM + r] = run_l;
-    named_bar_sync(1 + q, 64);
-    const float l_row = run_l + xmax[(half ^ 1) * kBM + r];
+    float l_row = run_l;
+    if constexpr (C::kWPQ == 2) {
+      xmax[half * kBM + r] = run_l;
+      named_bar_sync(1 + q, 64);
+      l_row += xmax[(half ^ 1) * kBM + r];
+    }
     const int tid = threadIdx.x - 64;     // 0..255 over the softmax warps
     constexpr int kF4 = DH / 4;           // float4 per row
     if (a.splits == 1) {

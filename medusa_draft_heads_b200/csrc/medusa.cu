@@ -716,8 +716,41 @@ struct AttnPlan {
   bool tc;                  // tensor-core path (the GQA group divides 128)
   int G, R, max_chunks;     // CUDA-core path
   int rtiles, splits, cps;  // tensor-core path
+  int ch;                   // tensor-core path: keys per chunk (64: two CTAs per SM; 128: one)
   size_t off_ml, off_cnt, bytes;
 };
+
+// Clusters of `cs` CTAs of the tensor-core attention kernel (head dim DH,
+// CH-key chunks) that can be resident at once (0 when none can be placed).
+template <int DH, int CH>
+int attn_max_clusters(int cs) {
+  static std::mutex mu;
+  static int cache[md::attn_tc::kMaxSplits + 1] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[cs] >= 0) return cache[cs];
+  using C = md::attn_tc::Cfg<DH, CH>;
+  auto kern = md::attn_tc::attn_tc_kernel<DH, CH>;
+  int n = 0;
+  if (set_smem(kern, C::kSmem) == MD_OK) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs, 64);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  cache[cs] = n;
+  return n;
+}
 
 AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
   using md::heads::align256;
@@ -730,17 +763,32 @@ AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
     // (Finer splits that even out unequal prefix lengths measured slower: every
     // CTA pays a prologue and epilogue of a few chunks' time and the merge.)
     p.rtiles = (p.R + 127) / 128;
-    const int chunks = (S_max + md::attn_tc::kBN - 1) / md::attn_tc::kBN;
     const int base = B * Hkv * p.rtiles;
-    int splits = std::max(1, num_sms() / base);
+    // Chunk size. 128-key chunks issue fewer MMAs per key and win while the
+    // tiles fit one wave of CTAs (70B, B = 1: 25 vs 31 us). Past one wave,
+    // 64-key chunks run two CTAs per SM (one CTA's prologue and split merge
+    // overlap the other's chunk loop), and win when they halve the waves
+    // enough: a two-CTA wave measured ~1.7 one-CTA waves (8B sweep, B = 32:
+    // 256 or 768 tiles, 8-18 % faster; B = 16 and the batched 70B, 320-384
+    // tiles, 2-11 % slower).
+    const int sms = num_sms();
+    const int waves128 = (base + sms - 1) / sms, waves64 = (base + 2 * sms - 1) / (2 * sms);
+    p.ch = (base > sms && 17 * waves64 < 10 * waves128) ? 64 : 128;
+    const int chunks = (S_max + p.ch - 1) / p.ch;
+    int splits = std::max(1, sms * (p.ch == 64 ? 2 : 1) / base);
     splits = std::min(std::min(splits, chunks), md::attn_tc::kMaxSplits);
+    // every tile's cluster resident at once (clusters must fit a GPC, so the
+    // cluster occupancy, not the SM count alone, bounds them)
+    if (p.ch == 64)
+      while (splits > 1 && (dh == 128 ? attn_max_clusters<128, 64>(splits) : attn_max_clusters<64, 64>(splits)) < base)
+        --splits;
     p.cps = (chunks + splits - 1) / splits;
     p.splits = (chunks + p.cps - 1) / p.cps;
     p.max_chunks = chunks;
     p.off_ml = p.off_cnt = 0;
     p.bytes = 256;          // the splits merge through distributed shared memory: no scratch
   } else {
-    p.rtiles = p.splits = p.cps = 0;
+    p.rtiles = p.splits = p.cps = p.ch = 0;
     p.max_chunks = (S_max + md::attn::kChunk - 1) / md::attn::kChunk;
     const size_t rows = size_t(B) * Hkv * p.max_chunks * p.R;
     p.off_ml = align256(rows * dh * 4);
@@ -749,7 +797,7 @@ AttnPlan attn_plan(int B, int T, int Hq, int Hkv, int dh, int S_max) {
   return p;
 }
 
-template <int DH>
+template <int DH, int CH>
 md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc, const md_bf16* vc,
                          const int32_t* prefix_len, int S_max, const md_tree* tree, int B, int Hq, int Hkv, float sc,
                          float* out, void* ws, cudaStream_t st) {
@@ -770,8 +818,8 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MD_ERR_CUDA;
   }
-  if ((s = make_map_3d_sw128(&kmap, kc, DH, S_max, uint64_t(B) * Hkv, 64, kBN)) != MD_OK) return s;
-  if ((s = make_map_3d_sw128(&vmap, vc, DH, S_max, uint64_t(B) * Hkv, 64, kBN)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&kmap, kc, DH, S_max, uint64_t(B) * Hkv, 64, CH)) != MD_OK) return s;
+  if ((s = make_map_3d_sw128(&vmap, vc, DH, S_max, uint64_t(B) * Hkv, 64, CH)) != MD_OK) return s;
   (void)ws;
   Args a;
   a.prefix_len = prefix_len;
@@ -779,12 +827,12 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   a.B = B; a.S_max = S_max; a.Hq = Hq; a.Hkv = Hkv; a.G = pl.G; a.R = pl.R; a.rtiles = pl.rtiles;
   a.splits = pl.splits; a.chunks_per_split = pl.cps;
   a.scale_log2 = sc * 1.4426950408889634f;
-  constexpr int sm = Cfg<DH>::kSmem;
-  if ((s = set_smem(attn_tc_kernel<DH>, sm)) != MD_OK) return s;
+  constexpr int sm = Cfg<DH, CH>::kSmem;
+  if ((s = set_smem(attn_tc_kernel<DH, CH>, sm)) != MD_OK) return s;
   // the KV splits of a tile form one cluster (they merge through its shared memory)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.splits, Hkv * pl.rtiles, B);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Cfg<DH, CH>::kThreads);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -796,7 +844,7 @@ md_status launch_attn_tc(const AttnPlan& pl, const md_bf16* q, const md_bf16* kc
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cuda_ok(cudaLaunchKernelEx(&cfg, attn_tc_kernel<DH>, qmap, kmap, vmap, tree->tp, a));
+  return cuda_ok(cudaLaunchKernelEx(&cfg, attn_tc_kernel<DH, CH>, qmap, kmap, vmap, tree->tp, a));
 }
 
 // ----------------------------- Hydra planning ------------------------------
@@ -1221,8 +1269,15 @@ md_status md_tree_attention(const md_bf16* q, const md_bf16* k_cache, const md_b
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(float(dh));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (pl.tc) {
-    return dh == 128 ? launch_attn_tc<128>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out, ws, st)
-                     : launch_attn_tc<64>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out, ws, st);
+    if (pl.ch == 64)
+      return dh == 128 ? launch_attn_tc<128, 64>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out,
+                                                 ws, st)
+                       : launch_attn_tc<64, 64>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out,
+                                                ws, st);
+    return dh == 128 ? launch_attn_tc<128, 128>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out,
+                                                ws, st)
+                     : launch_attn_tc<64, 128>(pl, q, k_cache, v_cache, prefix_len, S_max, tree, B, Hq, Hkv, sc, out,
+                                               ws, st);
   }
   md::attn::Args a;
   a.q = q; a.kc = k_cache; a.vc = v_cache; a.prefix_len = prefix_len;

@@ -97,6 +97,10 @@ def _attention_case(seed, tups, B, Hq, Hkv, dh, P, S_max, scale=0.0):
     ("long-ragged", ((10, 10, 10, 10), 64), 4, 32, 8, 128, [1024, 8191, 333, 5000]),
     # 9 row tiles per KV head (more than a portable cluster): one CTA per tile, no multicast
     ("g16-9tiles", ((10, 10, 10, 10), 64), 2, 16, 1, 64, [700, 2100]),
+    # more (request, KV head, row tile) tiles than one wave holds (160 and 768):
+    # 64-key chunks, two CTAs per SM
+    ("many-tiles-dh64", ((4, 3, 2, 2), 16), 40, 16, 4, 64, [int(x) for x in np.arange(40) * 37 % 400 + 60]),
+    ("many-tiles-dh128", ((10, 10, 10, 10), 64), 32, 32, 8, 128, [int(x) for x in np.arange(32) * 113 % 700 + 40]),
 ])
 def test_tree_attention_matches_oracle(name, tree, B, Hq, Hkv, dh, P):
     kph, n = tree
