@@ -540,13 +540,17 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
 // up to kmax entries. In "partitioned" mode slot c is CTA c of the kernel that
 // produced them (the CTAs that worked on row m): that kernel split `units`
 // work units, ordered (head, column tile of `ntiles`), into contiguous CTA
-// ranges, and only CTAs whose range touches head k wrote a list. Every list
-// is sorted and holds kk entries at or above its kk-th, so the head's top kk
-// lie at or above the best of the lists' kk-th entries: only entries at or
-// above that threshold (typically a few dozen of the few hundred) are
-// compacted into shared memory, padded to a power of two and bitonic-sorted in
-// the top-k order (value descending, then id ascending); the first kk are the
-// head's top-k.
+// ranges, so the slots that hold a list for head k form one contiguous range
+// [slot_lo[k], slot_hi[k]), which the host works out with the producer's own
+// partition arithmetic (set_merge_ranges). Every list is sorted, so the
+// head's top kk lie at or above two thresholds: the best of the lists' kk-th
+// entries (each list holds kk entries at or above its own), and the kk-th
+// best of the lists' first entries (kk distinct candidates reach it). Only
+// entries at or above the stricter one are kept: a few more than kk, where
+// the first threshold alone keeps hundreds when there are many lists. Each
+// kept entry's position in the top-k order (value descending, then id
+// ascending) is the number of kept entries ahead of it, counted in shared
+// memory; an entry whose position is below kk writes itself there.
 // ---------------------------------------------------------------------------
 struct MergeArgs {
   const float* cand_val;
@@ -558,69 +562,117 @@ struct MergeArgs {
   int stages;          // > 0: the producer cut units x stages items (stages per unit), not whole units
   int kh;              // heads for the top-k size: row mk uses kph[mk % kh]
   int kph[MD_MAX_K];
+  int slot_lo[MD_MAX_K], slot_hi[MD_MAX_K];   // slots holding head k's lists (set_merge_ranges)
 };
+
+// The slot range of each head. Slot c covered the producer's items
+// [c W / nslots, (c + 1) W / nslots) of W = units x stages (or whole units),
+// in the same 64-bit arithmetic as the producer; head k owns the items
+// [k ntiles S, (k + 1) ntiles S). Both ends are non-decreasing in c, so the
+// slots touching head k are contiguous.
+inline void set_merge_ranges(MergeArgs& a) {
+  for (int k = 0; k < MD_MAX_K; ++k) {
+    a.slot_lo[k] = 0;
+    a.slot_hi[k] = 0;
+  }
+  const long long S = a.stages > 0 ? a.stages : 1;
+  const long long W = (long long)a.units * S;
+  for (int k = 0; k < a.K && k < MD_MAX_K; ++k) {
+    if (!a.partitioned) {
+      a.slot_hi[k] = a.nslots;
+      continue;
+    }
+    int lo = a.nslots, hi = 0;
+    for (int c = 0; c < a.nslots; ++c) {
+      const long long w0 = a.stages > 0 ? (long long)c * W / a.nslots : (long long)c * a.units / a.nslots;
+      const long long w1 = a.stages > 0 ? (long long)(c + 1) * W / a.nslots : (long long)(c + 1) * a.units / a.nslots;
+      if (w1 > (long long)k * a.ntiles * S && w0 < (long long)(k + 1) * a.ntiles * S) {
+        lo = c < lo ? c : lo;
+        hi = c + 1;
+      }
+    }
+    a.slot_lo[k] = lo < hi ? lo : 0;
+    a.slot_hi[k] = lo < hi ? hi : 0;
+  }
+}
 
 constexpr int kMergeCap = 4096;          // candidates per (row, head): nslots * kmax <= kMergeCap
 constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kMergePer = kMergeCap / kMergeThreads;   // candidates per thread
+static_assert(kMergePer * kMergeWarps == 4 * 32, "the count scan gives each lane four counts");
 
 __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a) {
-  pdl_wait_primary();          // candidates come from the previous kernel
+  pdl_wait_primary();          // candidates come from the previous kernel (no-op in plain stream order)
   pdl_launch_dependents();
   __shared__ float sv[kMergeCap];
   __shared__ int si[kMergeCap];
-  __shared__ int slot_of[kMergeCap / 2];
-  __shared__ int warp_cnt[kMergeThreads / 32];
-  __shared__ int n_lists;
+  __shared__ int pass_cnt[kMergePer * kMergeWarps];   // [pass][warp]: kept counts, then offsets
+  __shared__ float red_v[kMergeWarps];
+  __shared__ int red_i[kMergeWarps];
+  __shared__ int n_keep;
+  __shared__ float head_v[kMergeThreads];      // each list's first entry
+  __shared__ int head_i[kMergeThreads];
+  __shared__ float first_v;                    // the kk-th best of them
+  __shared__ int first_i;
   const int mk = blockIdx.x;
   const int k = mk % a.K;
   const int kk = param_at(a.kph, mk % a.kh);
+  const int lo = param_at(a.slot_lo, k), hi = param_at(a.slot_hi, k);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t base = size_t(mk) * a.nslots * a.kmax;
-  if (threadIdx.x == 0) n_lists = 0;
-  __syncthreads();
+  const size_t base = (size_t(mk) * a.nslots + lo) * a.kmax;
+  const int n = (hi - lo) * kk;        // candidates: the first kk entries of each list
 
-  // 1. the slots that hold a list for head k, in slot order
-  for (int c0 = 0; c0 < a.nslots; c0 += kMergeThreads) {
-    const int c = c0 + threadIdx.x;
-    bool rel = c < a.nslots;
-    if (rel && a.partitioned) {
-      const long long S = a.stages > 0 ? a.stages : 1;     // items per unit
-      const long long W = (long long)a.units * S;
-      const long long w0 = a.stages > 0 ? (long long)c * W / a.nslots : (long long)c * a.units / a.nslots;
-      const long long w1 = a.stages > 0 ? (long long)(c + 1) * W / a.nslots : (long long)(c + 1) * a.units / a.nslots;
-      rel = w1 > (long long)k * a.ntiles * S && w0 < (long long)(k + 1) * a.ntiles * S;
+  // 1. every candidate this thread owns (e = pass * threads + thread) is
+  // loaded at once. Its list is e / kk, taken as floor((e + 1/2) / kk) in
+  // fp32: the quotient sits at least 1/(2 kk) >= 1/32 from an integer and
+  // its rounding error is below 4096 x 2^-23, so the floor is exact.
+  const float rkk = 1.0f / float(kk);
+  float cv[kMergePer];
+  int ci[kMergePer];
+  int lr[kMergePer];     // the candidate's place in its list (-1: none)
+  int li[kMergePer];     // its list
+#pragma unroll
+  for (int q = 0; q < kMergePer; ++q) {
+    const int e = q * kMergeThreads + threadIdx.x;
+    cv[q] = -INFINITY;
+    ci[q] = -1;
+    lr[q] = -1;
+    li[q] = 0;
+    if (e < n) {
+      const int l = __float2int_rd((float(e) + 0.5f) * rkk);
+      const int r = e - l * kk;
+      const size_t at = base + size_t(l) * a.kmax + r;
+      ci[q] = a.cand_id[at];
+      cv[q] = a.cand_val[at];
+      lr[q] = r;
+      li[q] = l;
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, rel);
-    if (lane == 0) warp_cnt[warp] = __popc(bal);
-    __syncthreads();
-    int off = n_lists;
-    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
-    if (rel) slot_of[off + __popc(bal & ((1u << lane) - 1))] = c;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int t = n_lists;
-      for (int w = 0; w < kMergeThreads / 32; ++w) t += warp_cnt[w];
-      n_lists = t;
-    }
-    __syncthreads();
   }
-  // 2. a threshold: each list holds kk entries at or above its own kk-th, so
-  // the head's top kk all lie at or above the best of the lists' kk-th
-  // entries; only those entries are sorted.
-  __shared__ float red_v[kMergeThreads / 32];
-  __shared__ int red_i[kMergeThreads / 32];
+
+  // 2. the threshold, the stricter of two that no member of the head's top
+  // kk falls below: (a) the best of the lists' kk-th entries (each list holds
+  // kk entries at or above its own kk-th); (b) the kk-th best of the lists'
+  // first entries (kk distinct candidates reach it). With many lists (a)
+  // alone keeps hundreds of entries, (b) a few more than kk.
+  const int n_lists = hi - lo;
+  const bool use_first = n_lists <= kMergeThreads;
+  if (threadIdx.x == 0) {
+    first_v = -INFINITY;
+    first_i = INT_MAX;
+  }
   {
     float bv = -INFINITY;
     int bi = INT_MAX;
-    for (int l = threadIdx.x; l < n_lists; l += kMergeThreads) {
-      const size_t at = base + size_t(slot_of[l]) * a.kmax + (kk - 1);
-      const int x = a.cand_id[at];
-      const float v = a.cand_val[at];
-      if (x >= 0) {
-        if (better(v, x, bv, bi)) {
-          bv = v;
-          bi = x;
-        }
+#pragma unroll
+    for (int q = 0; q < kMergePer; ++q) {
+      if (lr[q] == kk - 1 && ci[q] >= 0 && better(cv[q], ci[q], bv, bi)) {
+        bv = cv[q];
+        bi = ci[q];
+      }
+      if (lr[q] == 0 && use_first) {
+        head_v[li[q]] = ci[q] >= 0 ? cv[q] : -INFINITY;
+        head_i[li[q]] = ci[q] >= 0 ? ci[q] : INT_MAX;
       }
     }
 #pragma unroll
@@ -636,91 +688,110 @@ __global__ void __launch_bounds__(kMergeThreads) heads_merge_kernel(MergeArgs a)
       red_v[warp] = bv;
       red_i[warp] = bi;
     }
-    __syncthreads();
   }
+  __syncthreads();
   float tv = red_v[0];
   int ti = red_i[0];
 #pragma unroll
-  for (int w = 1; w < kMergeThreads / 32; ++w)
+  for (int w = 1; w < kMergeWarps; ++w)
     if (better(red_v[w], red_i[w], tv, ti)) {
       tv = red_v[w];
       ti = red_i[w];
     }
-
-  // 3. gather the (value, id) pairs at or above the threshold, in slot order;
-  // every candidate this thread looks at is loaded first, so the loads are in
-  // flight together instead of one dependent round trip per pass
-  constexpr int kPer = kMergeCap / kMergeThreads;
-  const int n = n_lists * kk;
-  float cv[kPer];
-  int ci[kPer];
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const int e = q * kMergeThreads + threadIdx.x;
-    cv[q] = -INFINITY;
-    ci[q] = -1;
-    if (e < n) {
-      const size_t at = base + size_t(slot_of[e / kk]) * a.kmax + e % kk;
-      ci[q] = a.cand_id[at];
-      cv[q] = a.cand_val[at];
+  // (b): list l's first entry is the kk-th best of the first entries when
+  // exactly kk - 1 of them are ahead of it (an identical pair counts as
+  // ahead when its list comes first, so the places are a permutation)
+  if (use_first && threadIdx.x < n_lists && head_i[threadIdx.x] != INT_MAX) {
+    const int t = threadIdx.x;
+    const float v = head_v[t];
+    const int x = head_i[t];
+    int place = 0;
+#pragma unroll 4
+    for (int j = 0; j < n_lists; ++j) {
+      const float vj = head_v[j];
+      const int xj = head_i[j];
+      place += (better(vj, xj, v, x) || (vj == v && xj == x && j < t)) ? 1 : 0;
+    }
+    if (place == kk - 1) {
+      first_v = v;
+      first_i = x;
     }
   }
-  // keep flags and per-warp counts of every pass, then one prefix: the order
-  // of the kept entries is the candidates' order e = q * threads + thread
-  __shared__ int pass_cnt[kPer][kMergeThreads / 32];
-  unsigned bal[kPer];
+  __syncthreads();
+  if (better(first_v, first_i, tv, ti)) {
+    tv = first_v;
+    ti = first_i;
+  }
+
+  // 3. keep the entries at or above the threshold: per-pass ballots, one
+  // exclusive scan of the (pass, warp) counts by warp 0, then each kept
+  // entry stores itself at its offset (the candidates' order)
+  unsigned bal[kMergePer];
 #pragma unroll
-  for (int q = 0; q < kPer; ++q) {
+  for (int q = 0; q < kMergePer; ++q) {
     const bool keep = ci[q] >= 0 && (better(cv[q], ci[q], tv, ti) || (cv[q] == tv && ci[q] == ti));
     bal[q] = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) pass_cnt[q][warp] = __popc(bal[q]);
+    if (lane == 0) pass_cnt[q * kMergeWarps + warp] = __popc(bal[q]);
   }
   __syncthreads();
-  int run = 0;
+  if (warp == 0) {
+    int c[4], s = 0;
 #pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    int off = run;
-    for (int w = 0; w < warp; ++w) off += pass_cnt[q][w];
+    for (int j = 0; j < 4; ++j) {
+      c[j] = pass_cnt[4 * lane + j];
+      s += c[j];
+    }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - s;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      pass_cnt[4 * lane + j] = run;
+      run += c[j];
+    }
+    if (lane == 31) n_keep = incl;
+  }
+  __syncthreads();
+  const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+  for (int q = 0; q < kMergePer; ++q)
     if ((bal[q] >> lane) & 1u) {
-      const int at = off + __popc(bal[q] & ((1u << lane) - 1));
+      const int at = pass_cnt[q * kMergeWarps + warp] + __popc(bal[q] & below);
       sv[at] = cv[q];
       si[at] = ci[q];
     }
-    for (int w = 0; w < kMergeThreads / 32; ++w) run += pass_cnt[q][w];
-  }
-  const int nk = run;
-  int N = 32;
-  while (N < nk) N <<= 1;
-  for (int e = nk + threadIdx.x; e < N; e += kMergeThreads) {   // pad with (-inf, INT_MAX)
-    sv[e] = -INFINITY;
-    si[e] = INT_MAX;
-  }
+  const int nk = n_keep;
   __syncthreads();
 
-  // 4. bitonic sort, best first
-  for (int size = 2; size <= N; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < (N >> 1); t += kMergeThreads) {
-        const int i = 2 * t - (t & (stride - 1));     // lower index of the pair
-        const int j = i + stride;
-        const bool desc = (i & size) == 0;            // this run is ordered best first
-        const float vi = sv[i], vj = sv[j];
-        const int ii = si[i], ij = si[j];
-        if (better(vj, ij, vi, ii) == desc) {
-          sv[i] = vj; si[i] = ij;
-          sv[j] = vi; si[j] = ii;
-        }
-      }
-      __syncthreads();
+  // 4. each kept entry's place is the number of kept entries ahead of it in
+  // the top-k order (an identical pair counts as ahead when it was stored
+  // earlier, so the places are a permutation). Sorted lists keep at most
+  // kk^2 <= 256 entries, one per thread: only the kk lists whose first entry
+  // reaches the threshold can hold an entry that does (or fewer than kk
+  // lists hold any); the loop covers any count all the same.
+  for (int t = threadIdx.x; t < nk; t += kMergeThreads) {
+    const float v = sv[t];
+    const int x = si[t];
+    int place = 0;
+#pragma unroll 4
+    for (int j = 0; j < nk; ++j) {
+      const float vj = sv[j];
+      const int xj = si[j];
+      place += (better(vj, xj, v, x) || (vj == v && xj == x && j < t)) ? 1 : 0;
+    }
+    if (place < kk) {
+      a.topk_vals[size_t(mk) * a.kmax + place] = v;
+      a.topk_ids[size_t(mk) * a.kmax + place] = x;
     }
   }
-
-  // 5. the first kk entries; the rest of the kmax slots are empty
-  if (threadIdx.x < a.kmax) {
-    const int r = threadIdx.x;
-    const bool used = r < kk && r < N && si[r] != INT_MAX;
-    a.topk_vals[size_t(mk) * a.kmax + r] = used ? sv[r] : -INFINITY;
-    a.topk_ids[size_t(mk) * a.kmax + r] = used ? si[r] : -1;
+  const int filled = nk < kk ? nk : kk;      // the rest of the kmax slots are empty
+  if (threadIdx.x >= filled && threadIdx.x < a.kmax) {
+    a.topk_vals[size_t(mk) * a.kmax + threadIdx.x] = -INFINITY;
+    a.topk_ids[size_t(mk) * a.kmax + threadIdx.x] = -1;
   }
 }
 

@@ -115,6 +115,17 @@ md_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, 
   return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
 }
 
+// The top-k merge is launched in plain stream order: as a dependent launch
+// its CTAs became resident beside the still-running projection kernel and
+// waited there, and the projection ran slower for it (a four-level Hydra
+// draft at 70B shapes took 1.50 ms that way against 1.46 ms in plain order).
+// The kernel's own griddepcontrol instructions are no-ops in this form, and
+// the launch after it can still be a dependent one.
+inline md_status launch_merge(const md::heads::MergeArgs& ma, int blocks, cudaStream_t st) {
+  md::heads::heads_merge_kernel<<<blocks, md::heads::kMergeThreads, 0, st>>>(ma);
+  return cuda_ok(cudaGetLastError());
+}
+
 template <typename Kernel>
 md_status set_smem(Kernel k, int bytes) {
   return cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
@@ -191,7 +202,8 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   ma.partitioned = 1; ma.units = pl.units; ma.ntiles = pl.ntiles; ma.kh = pl.K;
   ma.stages = va.stream_k ? pl.d / kStageRows : 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
-  return launch_pdl(heads_merge_kernel, dim3(pl.M * pl.K), dim3(256), 0, st, ma);
+  md::heads::set_merge_ranges(ma);
+  return launch_merge(ma, pl.M * pl.K, st);
 }
 
 // Workspace of the tensor-core path: z [K, M, d] bf16 and the candidates
@@ -356,7 +368,8 @@ md_status launch_heads_gemm(int M, int d, int V, int K, int kmax, const md_bf16*
   ma.partitioned = 1; ma.units = K * pl.ntiles2; ma.ntiles = pl.ntiles2; ma.kh = K;
   ma.stages = 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
-  return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
+  md::heads::set_merge_ranges(ma);
+  return launch_merge(ma, M * K, st);
 }
 
 // ---------------- tensor-core heads with the weights as M (2 .. 32 rows) ----------------
@@ -457,7 +470,8 @@ md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, 
   ma.partitioned = 1; ma.units = K * pl.nt2; ma.ntiles = pl.nt2; ma.kh = K;
   ma.stages = pl.S;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = a.kph[k];
-  return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
+  md::heads::set_merge_ranges(ma);
+  return launch_merge(ma, M * K, st);
 }
 
 // ------------------- shared vocabulary projection (one Wv) -------------------
@@ -559,7 +573,8 @@ md_status launch_heads_shared_skinny(const SharedPlan& sp, int M, int d, int V, 
   ma.partitioned = 1; ma.units = sp.nt2; ma.ntiles = sp.nt2; ma.kh = K;
   ma.stages = sp.S;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = a.kph[k];
-  return launch_pdl(md::heads::heads_merge_kernel, dim3(M * K), dim3(256), 0, st, ma);
+  md::heads::set_merge_ranges(ma);
+  return launch_merge(ma, M * K, st);
 }
 
 template <int MK>
@@ -622,7 +637,8 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   ma.partitioned = 1; ma.units = p2.units; ma.ntiles = p2.ntiles; ma.kh = p1.K;
   ma.stages = va.stream_k ? p2.d / kStageRows : 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = va.kph[k];
-  return launch_pdl(heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
+  md::heads::set_merge_ranges(ma);
+  return launch_merge(ma, MK, st);
 }
 
 template <int KK>
@@ -660,7 +676,8 @@ md_status launch_heads_shared_gemm(const SharedPlan& sp, int M, int d, int V, in
   ma.partitioned = 1; ma.units = sp.g2.ntiles2; ma.ntiles = sp.g2.ntiles2; ma.kh = K;
   ma.stages = 0;
   for (int k = 0; k < MD_MAX_K; ++k) ma.kph[k] = ga.kph[k];
-  return launch_pdl(md::heads::heads_merge_kernel, dim3(MK), dim3(256), 0, st, ma);
+  md::heads::set_merge_ranges(ma);
+  return launch_merge(ma, MK, st);
 }
 
 md_status heads_check(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax) {

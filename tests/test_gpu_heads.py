@@ -73,6 +73,30 @@ def test_topk_bit_exact_on_exact_integer_logits(M, d, V, kph):
     assert ties > 0
 
 
+@pytest.mark.parametrize("M,K,kk", [(1, 4, 10), (4, 4, 10), (40, 2, 16)])
+def test_topk_exact_when_most_candidates_pass_the_threshold(M, K, kk):
+    """Every 256-column tile holds kk - 1 columns of the top value: each list's
+    first kk - 1 entries tie at the top and its kk-th is lower, so the best of
+    the lists' kk-th entries lets hundreds of tied entries through and the
+    kk-th best of the lists' first entries (ties to the lower id) decides."""
+    d, V = 128, 256 * 32
+    rng = np.random.default_rng(40 + M)
+    hv = rng.choice(np.array([-1.0, 1.0], dtype=np.float32), size=d)
+    c = rng.integers(0, 2, (K, V)).astype(np.float32)
+    c[:, (np.arange(V) % 256) < kk - 1] = 3.0
+    h = gen.f32_to_bf16_bits(np.tile(hv, (M, 1)))
+    Wv = gen.f32_to_bf16_bits(hv[None, :, None] * c[:, None, :])     # logit = c * d exactly
+    W1 = np.zeros((K, d, d), dtype=np.uint16)
+    b1 = np.zeros((K, d), dtype=np.uint16)
+    kph = (kk,) * K
+    ids, vals, logits = _run(h, W1, b1, Wv, kph)
+    rid, rval, rlog, _ = oh.medusa_heads(h, W1, b1, Wv, kph)
+    assert np.array_equal(logits, rlog.astype(np.float32))
+    assert np.array_equal(ids, rid)
+    assert np.array_equal(vals, rval.astype(np.float32))
+    assert np.all(rval[:, :, kk - 1] == 3 * d)
+
+
 def test_heads_are_deterministic():
     h, W1, b1, Wv = head_weights(5, 512, 2048, 4, 2)
     a = _run(h, W1, b1, Wv, (10, 10, 10, 10))
