@@ -177,32 +177,18 @@ __global__ void __launch_bounds__(MD_MAX_T) accept_walk_kernel(const __grid_cons
   if (j < T && a.ysamp) {
     amax[j] = a.ysamp[size_t(b) * T + j];
   } else if (j < T) {
-    // the row's chunk summaries in chunk order, eight loaded at a time
-    const float4* p = reinterpret_cast<const float4*>(a.part + size_t(b * T + j) * a.nchunks * kPartFloats);
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-    Soft sm{-INFINITY, 0.f, 0.f};
-    for (int c0 = 0; c0 < a.nchunks; c0 += 8) {
-      float4 q[8];
-      float w[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c0 + u < a.nchunks) {
-          q[u] = p[2 * (c0 + u)];                       // best value, best id, m, S
-          w[u] = typical ? p[2 * (c0 + u) + 1].x : 0.f;   // W
-        }
+    const float* p = a.part + size_t(b * T + j) * a.nchunks * kPartFloats;
+    float bv = p[0];
+    int bi = __float_as_int(p[1]);
+    Soft sm{p[2], p[3], p[4]};
+    for (int c = 1; c < a.nchunks; ++c) {
+      const float* q = p + size_t(c) * kPartFloats;
+      const int qi = __float_as_int(q[1]);
+      if (better(q[0], qi, bv, bi)) {
+        bv = q[0];
+        bi = qi;
       }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c0 + u < a.nchunks) {
-          const int qi = __float_as_int(q[u].y);
-          if (better(q[u].x, qi, bv, bi)) {
-            bv = q[u].x;
-            bi = qi;
-          }
-          if (typical) sm = soft_merge(sm, Soft{q[u].z, q[u].w, w[u]});
-        }
-      }
+      if (typical) sm = soft_merge(sm, Soft{q[2], q[3], q[4]});
     }
     amax[j] = bi;
     if (typical) {
