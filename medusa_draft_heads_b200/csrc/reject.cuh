@@ -119,14 +119,30 @@ struct ClusterReduce {
 __device__ __forceinline__ float expw(float x, float mx, float scale) { return exp2f((x - mx) * scale); }
 
 // Load a row's slice into smem and turn it into e = exp((x - max) / tau);
-// returns (max over the row, sum of e over the row).
+// returns (max over the row, sum of e over the row). The slice arrives as one
+// bulk copy (a single DRAM round trip) when its address and length allow,
+// else through per-thread loads. Every thread of the block calls this with
+// the block's earlier reads of `s` finished (the caller's last reduction).
 __device__ __forceinline__ float2 load_exp_row(const float* row, float* s, int lo, int n, float scale,
-                                               ClusterReduce& cr) {
+                                               ClusterReduce& cr, uint64_t* bar, uint32_t& phase) {
   float mx = -INFINITY;
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    const float x = __ldg(row + lo + i);
-    s[i] = x;
-    mx = fmaxf(mx, x);
+  const float* src = row + lo;
+  const bool bulk = n > 0 && (n & 3) == 0 && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(s)) & 15) == 0;
+  if (bulk) {
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();             // the exp values written over s before
+      mbar_arrive_expect_tx(smem_u32(bar), uint32_t(n) * 4u);
+      bulk_load(smem_u32(s), src, uint32_t(n) * 4u, smem_u32(bar));
+    }
+    if (!mbar_wait(smem_u32(bar), phase)) set_status(MD_DEV_TIMEOUT);
+    phase ^= 1u;
+    for (int i = threadIdx.x; i < n; i += kThreads) mx = fmaxf(mx, s[i]);
+  } else {
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const float x = __ldg(src + i);
+      s[i] = x;
+      mx = fmaxf(mx, x);
+    }
   }
   mx = cr.run(mx, true);
   float sum = 0.f;
@@ -151,13 +167,20 @@ __global__ void __launch_bounds__(kThreads, 1) reject_accept_kernel(const __grid
   __shared__ int ch_node[MD_MAX_KMAX];       // children of the current node, by rank
   __shared__ float ch_p[MD_MAX_KMAX], ch_q[MD_MAX_KMAX];   // p(y) and q(y) of each child's token
   __shared__ int n_ch;
+  __shared__ __align__(8) uint64_t load_bar;  // completes each row slice's bulk copy
   ClusterReduce cr{warp_red, part, red_out, 0};
+  uint32_t load_phase = 0;
 
   const int crank = int(cluster_ctarank());
   const int b = blockIdx.y;
   const int lo = min(a.V, crank * a.slice), n = min(a.V, lo + a.slice) - lo;
   const float sc_t = 1.4426950408889634f * a.inv_tau;
   const float sc_q = 1.4426950408889634f * a.inv_tau_q;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&load_bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
   pdl_wait_primary();
   pdl_launch_dependents();
 
@@ -173,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) reject_accept_kernel(const __grid
   float A = 0.f, Bc = 1.f;                  // r = max(0, p - A q) / Bc over the walk at `node`
   for (;;) {
     const float* zrow = a.logits + (size_t(b) * a.T + node) * a.V;
-    const float2 zs = load_exp_row(zrow, se, lo, n, sc_t, cr);
+    const float2 zs = load_exp_row(zrow, se, lo, n, sc_t, cr, &load_bar, load_phase);
     const float inv_se = 1.f / zs.y;
     A = 0.f;
     Bc = 1.f;
@@ -200,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) reject_accept_kernel(const __grid
     if (has_child) {
       if (qdepth != depth) {
         const float* xrow = a.head_logits + (size_t(hrow) * a.Kh + depth) * a.V;
-        const float2 xs = load_exp_row(xrow, sq, lo, n, sc_q, cr);
+        const float2 xs = load_exp_row(xrow, sq, lo, n, sc_q, cr, &load_bar, load_phase);
         q_max = xs.x;
         q_sum = xs.y;
         qdepth = depth;

@@ -104,3 +104,10 @@ def sweep_8b(B: int, tree: str, prefix: int, mode: str = "greedy") -> Workload:
         kph, n = (10, 10, 10, 10), int(tree)
     return replace(LLAMA8B, name=f"sweep8b-B{B}-{tree}-P{prefix}-{mode}", B=B, k_per_head=kph,
                    n_nodes=n, prefix=(prefix, prefix), logit_sigma=3.0, bump=3.0, mode=mode)
+
+
+# Profiling case for the 64-key, two-CTA-per-SM attention shape: the 8B sweep's
+# B = 32 point with the 64-node tree and a 1024-token prefix (768 row tiles,
+# more than one wave of 128-key CTAs).
+PROF_ATTN_B32 = replace(sweep_8b(32, "64", 1024), name="prof-attn-8b-b32")
+WORKLOADS[PROF_ATTN_B32.name] = PROF_ATTN_B32
