@@ -114,6 +114,10 @@ struct ClusterReduce {
   }
 };
 
+// Orders this thread's earlier generic-proxy shared-memory accesses (after a
+// block barrier: the block's) before later async-proxy (bulk copy) writes.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // e = exp2((x - mx) * scale) with scale = log2(e) / tau: the one formula used
 // for the slices and for single entries, so both give the same bits.
 __device__ __forceinline__ float expw(float x, float mx, float scale) { return exp2f((x - mx) * scale); }
