@@ -433,17 +433,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
             }
           } else {
-            // the unit's parts, summed in CTA order
+            // the unit's parts, summed in CTA order; two parts' loads in flight at once
 #pragma unroll
             for (int i = 0; i < kChunk; ++i) v0[i] = v1[i] = 0.f;
-            for (int c = cf; c <= cl; ++c) {
-              const int sl = range_lo(W, G, c) >= (long long)unit * S ? 0 : 1;
-              const float* pp = a.part + (size_t(c) * 2 + sl) * a.M * kTile + size_t(ch) * kChunk * kTile;
+            for (int c = cf; c <= cl; c += 2) {
+              const bool two = c + 1 <= cl;
+              const int sl0 = range_lo(W, G, c) >= (long long)unit * S ? 0 : 1;
+              const int sl1 = two && range_lo(W, G, c + 1) >= (long long)unit * S ? 0 : 1;
+              const float* pp0 = a.part + (size_t(c) * 2 + sl0) * a.M * kTile + size_t(ch) * kChunk * kTile;
+              const float* pp1 = a.part + (size_t(two ? c + 1 : c) * 2 + sl1) * a.M * kTile + size_t(ch) * kChunk * kTile;
+              float x0[kChunk], x1[kChunk], y0[kChunk], y1[kChunk];
 #pragma unroll
               for (int i = 0; i < kChunk; ++i) {
-                if (ch * kChunk + i < a.M) {
-                  v0[i] += __ldcg(pp + i * kTile + col0);
-                  v1[i] += __ldcg(pp + i * kTile + col0 + 128);
+                const bool live = ch * kChunk + i < a.M;
+                x0[i] = live ? __ldcg(pp0 + i * kTile + col0) : 0.f;
+                x1[i] = live ? __ldcg(pp0 + i * kTile + col0 + 128) : 0.f;
+                y0[i] = live && two ? __ldcg(pp1 + i * kTile + col0) : 0.f;
+                y1[i] = live && two ? __ldcg(pp1 + i * kTile + col0 + 128) : 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < kChunk; ++i) {
+                v0[i] += x0[i];
+                v1[i] += x1[i];
+                if (two) {
+                  v0[i] += y0[i];
+                  v1[i] += y1[i];
                 }
               }
             }
