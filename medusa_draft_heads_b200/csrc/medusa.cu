@@ -684,8 +684,9 @@ md_status heads_check(int32_t M, int32_t d, int32_t V, int32_t K, int32_t kmax) 
   if (M <= 0 || d <= 0 || V <= 0 || K <= 0 || kmax <= 0) return MD_ERR_INVALID_ARG;
   if (K > MD_MAX_K || kmax > MD_MAX_KMAX) return MD_ERR_UNSUPPORTED;
   if (M > md::gemm::kMaxM) return MD_ERR_UNSUPPORTED;
-  // the merge holds every candidate list of one (row, head) in shared memory
-  if (num_sms() > md::heads::kMergeCap / 2 || num_sms() * kmax > md::heads::kMergeCap) return MD_ERR_UNSUPPORTED;
+  // the merge loads every candidate of one (row, head) at once: at most one
+  // list of kmax entries per producer CTA, and producers run one CTA per SM
+  if (num_sms() * kmax > md::heads::kMergeCap) return MD_ERR_UNSUPPORTED;
   if (d % 64 != 0 || V % 8 != 0 || V < 256) return MD_ERR_UNSUPPORTED;
   if (size_t(K) * d >= (size_t(1) << 31) || V >= (1 << 30)) return MD_ERR_UNSUPPORTED;
   return MD_OK;
