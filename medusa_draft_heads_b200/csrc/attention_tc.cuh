@@ -137,6 +137,29 @@ __global__ void __launch_bounds__(Cfg<DH, CH>::kThreads, Cfg<DH, CH>::kMinBlocks
   const int split = blockIdx.x, rt = blockIdx.y % a.rtiles, hk = blockIdx.y / a.rtiles;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = tp.T;
+  // Set-up that reads no input (mbarriers, TMEM) runs before the wait for the
+  // previous kernel, overlapping its tail.
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&p_full[i]), kSoftWarps);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&o_full[i]), 1);
+    mbar_init(smem_u32(o_last), 1);
+    mbar_init(smem_u32(mma_done), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
   pdl_wait_primary();          // inputs may come from earlier kernels
   pdl_launch_dependents();
   // Blocks are launched in index order, so blockIdx.z walks the requests from
@@ -164,27 +187,6 @@ __global__ void __launch_bounds__(Cfg<DH, CH>::kThreads, Cfg<DH, CH>::kMinBlocks
   const int nch = max(0, c_end - c_begin);
   if (bad && split == 0 && blockIdx.y == 0 && threadIdx.x == 0) set_status(MD_DEV_BAD_PREFIX);
 
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(q_full), 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&k_full[i]), 1);
-      mbar_init(smem_u32(&k_empty[i]), 1);
-      mbar_init(smem_u32(&v_full[i]), 1);
-      mbar_init(smem_u32(&v_empty[i]), 1);
-    }
-    for (int i = 0; i < kSBufs; ++i) {
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&p_full[i]), kSoftWarps);
-    }
-    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&o_full[i]), 1);
-    mbar_init(smem_u32(o_last), 1);
-    mbar_init(smem_u32(mma_done), 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
