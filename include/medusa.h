@@ -229,7 +229,9 @@ MD_API md_status md_medusa_heads_sampled(const md_bf16* h, const md_bf16* W1, co
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
  *   first call before any stream capture on the device.
  * - Every call on a device shares the one array and leaves its contents
- *   behind; the call clears what must start at zero itself. Two calls whose
+ *   behind; the call clears what must start at zero itself (the one-row
+ *   streaming path needs nothing cleared: its tickets carry a per-call
+ *   epoch). Two calls whose
  *   kernels overlap on the GPU (different streams, no ordering between them)
  *   race on the array and give undefined results: order them on one stream
  *   or with events.

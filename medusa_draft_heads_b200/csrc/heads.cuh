@@ -77,7 +77,7 @@ inline Plan make_plan(int M, int d, int V, int K, int kmax, int num_sms) {
   size_t o = 0;
   p.off_zt = o;   o = align256(o + size_t(K) * d * kZPad * 2);
   p.off_part = o; o = align256(o + size_t(splits) * K * M * d * 4);
-  p.off_cnt = o;  o = align256(o + size_t(K) * p.ntile_o * 4);
+  p.off_cnt = o;  o = align256(o + size_t(K) * p.ntile_o * 8);      // epoch tickets (epoch_arrive)
   p.grid = std::min(num_sms, p.units);
   // Whole units over the CTAs leave a tail when they do not divide evenly
   // (2004 units of a 70B call over 148 CTAs: 13 or 14 each; 501 for one head:
@@ -85,12 +85,33 @@ inline Plan make_plan(int M, int d, int V, int K, int kmax, int num_sms) {
   // instead: a unit then spans at most two CTAs, whose partial logits the
   // second to finish adds up.
   p.stream_k = (p.units > p.grid && p.units % p.grid != 0) ? 1 : 0;
-  p.off_tick = o; o = align256(o + size_t(p.units) * 4);            // one ticket per unit (zeroed with the counters)
+  p.off_tick = o; o = align256(o + size_t(p.units) * 8);            // one epoch ticket per unit
   p.off_spart = o; o = align256(o + size_t(p.grid) * 2 * M * kTileV * 4);
   p.off_cval = o; o = align256(o + size_t(M) * K * p.grid * kmax * 4);
   p.off_cid = o;  o = align256(o + size_t(M) * K * p.grid * kmax * 4);
   p.bytes = o;
   return p;
+}
+
+// ---------------------------------------------------------------------------
+// Tickets that need no clearing between calls. A ticket word holds a call's
+// epoch (high 32 bits; every call of these kernels draws a new nonzero one on
+// the host) and that call's arrivals so far (low 32 bits). An arrival that
+// finds another epoch there (an earlier call's, zero, or whatever the
+// workspace held) starts the count afresh. Returns this arrival's index
+// within the call (0, 1, ...). The loop only retries while other CTAs of the
+// call are arriving at the same word, so it ends after at most as many
+// rounds as there are arrivals.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t epoch_arrive(unsigned long long* p, uint32_t epoch) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(p);
+  for (;;) {
+    const unsigned long long want =
+        uint32_t(cur >> 32) == epoch ? cur + 1ull : ((unsigned long long)epoch << 32) | 1ull;
+    const unsigned long long prev = atomicCAS(p, cur, want);
+    if (prev == cur) return uint32_t(want) - 1u;
+    cur = prev;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -106,8 +127,9 @@ struct W1Args {
   const uint16_t* b1;  // [K, d]
   uint16_t* zt;        // [K, d, 8]
   float* part;         // [splits, K, M, d]
-  int* counters;       // [K, ntile_o]
+  unsigned long long* counters;   // [K, ntile_o] epoch tickets (epoch_arrive)
   int d, K, splits, rows, ntile_o;
+  uint32_t epoch;      // this call's epoch
   int shared;          // 1: one projection for all heads: z row (m, k) goes to slot m*K + k of zt[0]
 };
 
@@ -119,7 +141,7 @@ __global__ void __launch_bounds__(kW1Threads, w1_blocks_per_sm(M)) heads_w1_kern
   __shared__ int is_last;
 
   pdl_launch_dependents();
-  pdl_wait_primary();   // h and the counters may come from the work before (dependent launch)
+  pdl_wait_primary();   // h may come from the work before (dependent launch)
 
   const int k = blockIdx.z, s = blockIdx.y, ct = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -206,8 +228,8 @@ __global__ void __launch_bounds__(kW1Threads, w1_blocks_per_sm(M)) heads_w1_kern
   __threadfence();
   __syncthreads();
   if (t == 0) {
-    const int ticket = atomicAdd(&a.counters[k * a.ntile_o + ct], 1);
-    is_last = (ticket == a.splits - 1);
+    const uint32_t ticket = epoch_arrive(&a.counters[k * a.ntile_o + ct], a.epoch);
+    is_last = (ticket == uint32_t(a.splits - 1));
   }
   __syncthreads();
   if (!is_last) return;
@@ -236,7 +258,6 @@ __global__ void __launch_bounds__(kW1Threads, w1_blocks_per_sm(M)) heads_w1_kern
                      zv[4] | (uint32_t(zv[5]) << 16), zv[6] | (uint32_t(zv[7]) << 16));
     }
   }
-  if (t == 0) a.counters[k * a.ntile_o + ct] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -258,7 +279,8 @@ struct VocabArgs {
   const float* gumbel_u;  // [M, K, V] uniforms (sampled drafts) or null (top-k of the logits)
   float inv_tau;          // 1 / draft temperature (sampled drafts)
   int stream_k;           // CTA ranges in (unit, stage) items instead of whole units
-  int* tickets;           // [units], zero at launch: a split unit's second finisher adds the parts
+  unsigned long long* tickets;   // [units] epoch tickets: a split unit's second finisher adds the parts
+  uint32_t epoch;         // this call's epoch
   float* spart;           // [gridDim.x][2][M][256]: partial logits of the units a CTA range cuts
   int d, V, K, kmax, ntiles, units, nstages;
   int shared, kh;      // shared projection: K == 1 and row m is (m / kh, head m % kh)
@@ -437,7 +459,7 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, 1)
       for (int m = 0; m < M; ++m) mine[m * kTileV + t] = v[m];
       __threadfence();
       named_bar_sync(1, kConsumerWarps * 32);
-      if (t == 0) s_ticket = atomicAdd(&a.tickets[unit], 1);
+      if (t == 0) s_ticket = int(epoch_arrive(&a.tickets[unit], a.epoch));
       named_bar_sync(1, kConsumerWarps * 32);
       fold = s_ticket == 1;
       if (fold) {

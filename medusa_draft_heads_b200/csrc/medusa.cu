@@ -133,9 +133,21 @@ md_status set_smem(Kernel k, int bytes) {
 
 // ----------------------------- heads launchers -----------------------------
 
-// zeroed: the workspace's counters and tickets are already zero (cleared by
-// the caller earlier on the stream), so no memset separates this call from
-// the kernel before it and the first kernel is launched dependent on it.
+// One epoch per call of the streaming heads kernels: their tickets carry it
+// (epoch_arrive), so the workspace needs no clearing between calls and the
+// first kernel is launched dependent on the kernel before it. Never 0, so
+// zeroed memory holds no epoch.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> counter{0};
+  uint32_t e;
+  do {
+    e = counter.fetch_add(1, std::memory_order_relaxed) + 1u;
+  } while (e == 0);
+  return e;
+}
+
+// zeroed: kept for the callers' uniformity; the streaming tickets need no
+// clearing (next_epoch).
 template <int M>
 md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
                        const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
@@ -147,21 +159,16 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   wa.h = h; wa.W1 = W1; wa.b1 = b1;
   wa.zt = reinterpret_cast<uint16_t*>(ws + pl.off_zt);
   wa.part = reinterpret_cast<float*>(ws + pl.off_part);
-  wa.counters = reinterpret_cast<int*>(ws + pl.off_cnt);
+  wa.counters = reinterpret_cast<unsigned long long*>(ws + pl.off_cnt);
   wa.d = pl.d; wa.K = pl.K; wa.splits = pl.splits; wa.rows = pl.rows; wa.ntile_o = pl.ntile_o;
   wa.shared = 0;
-  // phase-1 counters and phase-2 tickets are contiguous: one memset
-  if (!zeroed && (s = cuda_ok(cudaMemsetAsync(wa.counters, 0, pl.off_spart - pl.off_cnt, st))) != MD_OK) return s;
+  wa.epoch = next_epoch();
+  (void)zeroed;
   const int w1_smem = pl.rows * 16 + kConsumerWarps * M * kW1TileO * 4;
   if ((s = set_smem(heads_w1_kernel<M>, w1_smem)) != MD_OK) return s;
-  if (zeroed) {
-    if ((s = launch_pdl(heads_w1_kernel<M>, dim3(pl.ntile_o, pl.splits, pl.K), dim3(kW1Threads), w1_smem, st,
-                        wa)) != MD_OK)
-      return s;
-  } else {
-    heads_w1_kernel<M><<<dim3(pl.ntile_o, pl.splits, pl.K), kW1Threads, w1_smem, st>>>(wa);
-    if ((s = last_launch()) != MD_OK) return s;
-  }
+  if ((s = launch_pdl(heads_w1_kernel<M>, dim3(pl.ntile_o, pl.splits, pl.K), dim3(kW1Threads), w1_smem, st, wa)) !=
+      MD_OK)
+    return s;
 
   // phase 2 (programmatic dependent launch: its TMA of Wv may start before phase 1 ends)
   CUtensorMap map;
@@ -174,7 +181,8 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   va.gumbel_u = gumbel_u;
   va.inv_tau = inv_tau;
   va.stream_k = pl.stream_k;
-  va.tickets = reinterpret_cast<int*>(ws + pl.off_tick);
+  va.tickets = reinterpret_cast<unsigned long long*>(ws + pl.off_tick);
+  va.epoch = wa.epoch;
   va.spart = reinterpret_cast<float*>(ws + pl.off_spart);
   va.d = pl.d; va.V = pl.V; va.K = pl.K; va.kmax = pl.kmax; va.ntiles = pl.ntiles; va.units = pl.units;
   va.nstages = pl.nstages;
@@ -589,17 +597,14 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   wa.h = h; wa.W1 = W1; wa.b1 = b1;
   wa.zt = reinterpret_cast<uint16_t*>(ws + p1.off_zt);
   wa.part = reinterpret_cast<float*>(ws + p1.off_part);
-  wa.counters = reinterpret_cast<int*>(ws + p1.off_cnt);
+  wa.counters = reinterpret_cast<unsigned long long*>(ws + p1.off_cnt);
   wa.d = p1.d; wa.K = p1.K; wa.splits = p1.splits; wa.rows = p1.rows; wa.ntile_o = p1.ntile_o;
   wa.shared = 1;
-  if ((s = cuda_ok(cudaMemsetAsync(wa.counters, 0, size_t(p1.K) * p1.ntile_o * 4, st))) != MD_OK) return s;
-  // phase-2 tickets of the shared projection (its own plan p2)
-  if ((s = cuda_ok(cudaMemsetAsync(ws + sp.off2 + sp.tick2, 0, size_t(p2.units) * 4, st))) != MD_OK) return s;
+  wa.epoch = next_epoch();     // phase-1 counters and the shared projection's tickets (its own plan p2)
   auto run_w1 = [&](auto kern, int smem) -> md_status {
     md_status r;
     if ((r = set_smem(kern, smem)) != MD_OK) return r;
-    kern<<<dim3(p1.ntile_o, p1.splits, p1.K), kW1Threads, smem, st>>>(wa);
-    return last_launch();
+    return launch_pdl(kern, dim3(p1.ntile_o, p1.splits, p1.K), dim3(kW1Threads), smem, st, wa);
   };
   switch (M) {   // phase-1 rows (M * K <= 4)
     case 1: s = run_w1(heads_w1_kernel<1>, p1.rows * 16 + kConsumerWarps * 1 * kW1TileO * 4); break;
@@ -619,7 +624,8 @@ md_status launch_heads_shared_stream(const SharedPlan& sp, int M, const md_bf16*
   va.gumbel_u = nullptr;
   va.inv_tau = 1.f;
   va.stream_k = p2.stream_k;
-  va.tickets = reinterpret_cast<int*>(ws + sp.off2 + sp.tick2);
+  va.tickets = reinterpret_cast<unsigned long long*>(ws + sp.off2 + sp.tick2);
+  va.epoch = wa.epoch;
   va.spart = reinterpret_cast<float*>(ws + sp.off2 + sp.spart2);
   va.d = p2.d; va.V = p2.V; va.K = 1; va.kmax = p2.kmax; va.ntiles = p2.ntiles; va.units = p2.units;
   va.nstages = p2.nstages;
@@ -927,11 +933,8 @@ md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPl
 void heads_zero_range(int M, int d, int V, int K, int kmax, size_t* off, size_t* bytes) {
   *off = 0;
   *bytes = 0;
-  if (stream_rows(M)) {
-    const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
-    *off = pl.off_cnt;
-    *bytes = pl.off_spart - pl.off_cnt;
-  } else if (skinny_rows(M)) {
+  // the one-row streaming path's tickets carry a per-call epoch: nothing to clear
+  if (skinny_rows(M)) {
     const SkinnyPlan pl = skinny_plan(M, d, V, K, kmax);
     *off = pl.off_tick;
     *bytes = size_t(K) * (pl.nt1 + pl.nt2) * 4;

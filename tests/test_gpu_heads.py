@@ -97,6 +97,36 @@ def test_topk_exact_when_most_candidates_pass_the_threshold(M, K, kk):
     assert np.all(rval[:, :, kk - 1] == 3 * d)
 
 
+@pytest.mark.parametrize("fill", ["zeros", "ones", "random"])
+def test_streaming_heads_need_no_cleared_workspace(fill):
+    """The one-row path's tickets carry a per-call epoch: a workspace holding
+    anything at all, and the same workspace reused call after call, give the
+    same results bit for bit (several cut units and split-K tiles)."""
+    import medusa_draft_heads_b200 as md
+    M, d, V, kph = 1, 1024, 10000, (10, 4, 7, 1)      # 160 units over 148 CTAs: cut units
+    h, W1, b1, Wv = head_weights(77, d, V, len(kph), M)
+    ref_ids, ref_vals, ref_log = _run(h, W1, b1, Wv, kph)
+    K, kmax = len(kph), max(kph)
+    ws = md.workspace(md.heads_workspace_bytes(M, d, V, K, kmax))
+    if fill == "zeros":
+        ws.zero_()
+    elif fill == "ones":
+        ws.fill_(255)
+    else:
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda"))
+    hb, W1b, b1b, Wvb = bf16_tensor(h), bf16_tensor(W1), bf16_tensor(b1), bf16_tensor(Wv)
+    for _ in range(3):
+        ids = torch.full((M, K, kmax), -7, dtype=torch.int32, device="cuda")
+        vals = torch.zeros((M, K, kmax), dtype=torch.float32, device="cuda")
+        logits = torch.zeros((M, K, V), dtype=torch.float32, device="cuda")
+        md.medusa_heads(hb, W1b, b1b, Wvb, kph, ids, vals, ws, logits_dbg=logits)
+        torch.cuda.synchronize()
+        assert md.device_status() == 0
+        assert np.array_equal(ids.cpu().numpy(), ref_ids)
+        assert np.array_equal(vals.cpu().numpy(), ref_vals)
+        assert np.array_equal(logits.cpu().numpy(), ref_log)
+
+
 def test_heads_are_deterministic():
     h, W1, b1, Wv = head_weights(5, 512, 2048, 4, 2)
     a = _run(h, W1, b1, Wv, (10, 10, 10, 10))
