@@ -35,6 +35,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "heads.cuh"   // epoch_arrive
 
 namespace md {
 namespace skinny {
@@ -70,7 +71,8 @@ struct Args {
   int NRz;               // rows of each z matrix (the phase-2 row padding)
   int zg_mk;             // phase 1: row m of head k goes to row m * Kh + k of z[0] (shared projection)
   float* part;           // [gridDim.x][2][M][256]: partial sums of the units a CTA range cuts
-  int* tickets;          // [units], zero at launch
+  unsigned long long* tickets;   // [units] epoch tickets (md::heads::epoch_arrive)
+  uint32_t epoch;        // this call's epoch
   float* cand_val;       // phase 2: [M, Kh, gridDim.x, kmax], one list per (row, head, CTA)
   int* cand_id;
   float* logits_dbg;     // phase 2: [M, Kh, N] or null
@@ -414,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
         __threadfence();
         named_bar_sync(1, 128);
-        if (et == 0) s_ticket[buf] = atomicAdd(&a.tickets[unit], 1);
+        if (et == 0) s_ticket[buf] = int(md::heads::epoch_arrive(&a.tickets[unit], a.epoch));
         named_bar_sync(1, 128);
         cf = cta_of(W, G, (long long)unit * S);
         cl = cta_of(W, G, (long long)unit * S + S - 1);

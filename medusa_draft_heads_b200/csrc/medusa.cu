@@ -146,12 +146,10 @@ uint32_t next_epoch() {
   return e;
 }
 
-// zeroed: kept for the callers' uniformity; the streaming tickets need no
-// clearing (next_epoch).
 template <int M>
 md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf16* W1, const md_bf16* b1,
                        const md_bf16* Wv, const int32_t* kph, int32_t* topk_ids, float* topk_vals, float* logits_dbg,
-                       const float* gumbel_u, float inv_tau, uint8_t* ws, cudaStream_t st, bool zeroed = false) {
+                       const float* gumbel_u, float inv_tau, uint8_t* ws, cudaStream_t st) {
   using namespace md::heads;
   md_status s;
   // phase 1
@@ -163,7 +161,6 @@ md_status launch_heads(const md::heads::Plan& pl, const md_bf16* h, const md_bf1
   wa.d = pl.d; wa.K = pl.K; wa.splits = pl.splits; wa.rows = pl.rows; wa.ntile_o = pl.ntile_o;
   wa.shared = 0;
   wa.epoch = next_epoch();
-  (void)zeroed;
   const int w1_smem = pl.rows * 16 + kConsumerWarps * M * kW1TileO * 4;
   if ((s = set_smem(heads_w1_kernel<M>, w1_smem)) != MD_OK) return s;
   if ((s = launch_pdl(heads_w1_kernel<M>, dim3(pl.ntile_o, pl.splits, pl.K), dim3(kW1Threads), w1_smem, st, wa)) !=
@@ -410,7 +407,7 @@ SkinnyPlan skinny_plan(int M, int d, int V, int K, int kmax) {
   size_t o = 0;
   p.off_z = o;    o = align256(o + size_t(K) * p.NR * d * 2);
   p.off_part = o; o = align256(o + size_t(std::max(p.G1, p.G2)) * 2 * M * md::skinny::kTile * 4);
-  p.off_tick = o; o = align256(o + size_t(K) * (p.nt1 + p.nt2) * 4);
+  p.off_tick = o; o = align256(o + size_t(K) * (p.nt1 + p.nt2) * 8);   // epoch tickets
   p.off_cval = o; o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
   p.off_cid = o;  o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
   p.bytes = o;
@@ -441,7 +438,7 @@ template <int NR>
 md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, int kmax, const md_bf16* h,
                               const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, const int32_t* kph,
                               int32_t* topk_ids, float* topk_vals, float* logits_dbg, const float* gumbel_u,
-                              float inv_tau, uint8_t* ws, cudaStream_t st, bool zeroed = false) {
+                              float inv_tau, uint8_t* ws, cudaStream_t st) {
   using namespace md::skinny;
   md_status s;
   Args a = {};
@@ -450,16 +447,16 @@ md_status launch_heads_skinny(const SkinnyPlan& pl, int M, int d, int V, int K, 
   a.z = reinterpret_cast<uint16_t*>(ws + pl.off_z);
   a.NRz = NR; a.zg_mk = 0;
   a.part = reinterpret_cast<float*>(ws + pl.off_part);
-  int* tick = reinterpret_cast<int*>(ws + pl.off_tick);
+  unsigned long long* tick = reinterpret_cast<unsigned long long*>(ws + pl.off_tick);
+  a.epoch = next_epoch();      // both phases' tickets (distinct words): nothing to clear
   for (int k = 0; k < MD_MAX_K; ++k) a.kph[k] = k < K ? kph[k] : 0;
-  if (!zeroed && (s = cuda_ok(cudaMemsetAsync(tick, 0, size_t(K) * (pl.nt1 + pl.nt2) * 4, st))) != MD_OK) return s;
 
   // phase 1: z = bf16(h + SiLU(h W1_k + b1_k)) -- W1_k^T as the MMA's A, h^T as its B
   CUtensorMap wmap, xmap;
   if ((s = make_map_3d_sw128(&wmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&xmap, h, d, M, 1, kBK, NR)) != MD_OK) return s;
   a.N = d; a.ntiles = pl.nt1; a.tickets = tick;
-  if ((s = launch_skinny<EPI_SILU, NR>(wmap, xmap, a, pl.G1, zeroed, st)) != MD_OK) return s;
+  if ((s = launch_skinny<EPI_SILU, NR>(wmap, xmap, a, pl.G1, true, st)) != MD_OK) return s;
 
   // phase 2: logits = z_k Wv_k, running top-k per (row, head, CTA)
   if ((s = make_map_3d_sw128(&wmap, Wv, V, d, K, 64, kBK)) != MD_OK) return s;
@@ -516,7 +513,7 @@ SharedPlan shared_plan(int M, int d, int V, int K, int kmax) {
     size_t o = 0;
     p.off_z = o;    o = align256(o + size_t(p.NR2) * d * 2);
     p.off_part = o; o = align256(o + size_t(std::max(p.G1, p.G2)) * 2 * (M * K) * md::skinny::kTile * 4);
-    p.off_tick = o; o = align256(o + size_t(K * p.nt1 + p.nt2) * 4);
+    p.off_tick = o; o = align256(o + size_t(K * p.nt1 + p.nt2) * 8);   // epoch tickets
     p.off_cval = o; o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
     p.off_cid = o;  o = align256(o + size_t(M) * K * p.G2 * kmax * 4);
     p.bytes = o;
@@ -555,15 +552,15 @@ md_status launch_heads_shared_skinny(const SharedPlan& sp, int M, int d, int V, 
   a.z = reinterpret_cast<uint16_t*>(ws + sp.off_z);
   a.NRz = NR2; a.zg_mk = 1;
   a.part = reinterpret_cast<float*>(ws + sp.off_part);
-  int* tick = reinterpret_cast<int*>(ws + sp.off_tick);
+  unsigned long long* tick = reinterpret_cast<unsigned long long*>(ws + sp.off_tick);
+  a.epoch = next_epoch();      // both phases' tickets (distinct words): nothing to clear
   for (int k = 0; k < MD_MAX_K; ++k) a.kph[k] = k < K ? kph[k] : 0;
-  if ((s = cuda_ok(cudaMemsetAsync(tick, 0, size_t(K * sp.nt1 + sp.nt2) * 4, st))) != MD_OK) return s;
 
   CUtensorMap wmap, xmap;
   if ((s = make_map_3d_sw128(&wmap, W1, d, d, K, 64, kBK)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&xmap, h, d, M, 1, kBK, NR1)) != MD_OK) return s;
   a.M = M; a.Kh = K; a.N = d; a.ntiles = sp.nt1; a.tickets = tick; a.kh = 0;
-  if ((s = launch_skinny<EPI_SILU, NR1>(wmap, xmap, a, sp.G1, false, st)) != MD_OK) return s;
+  if ((s = launch_skinny<EPI_SILU, NR1>(wmap, xmap, a, sp.G1, true, st)) != MD_OK) return s;
 
   if ((s = make_map_3d_sw128(&wmap, Wv, V, d, 1, 64, kBK)) != MD_OK) return s;
   if ((s = make_map_3d_sw128(&xmap, a.z, d, NR2, 1, kBK, NR2)) != MD_OK) return s;
@@ -883,7 +880,7 @@ struct HydraPlan {
   int8_t slot[MD_MAX_T];              // node -> index among its depth's nodes with children (-1: none)
   int8_t node[MD_MAX_K][MD_MAX_T];    // level l, index q -> node
   size_t heads_bytes[MD_MAX_K];       // heads workspace of each level (its own region: the
-  size_t off_heads[MD_MAX_K];         // counters of every level are cleared once, up front)
+  size_t off_heads[MD_MAX_K];         // each level's heads workspace
   size_t off_x, off_ids, off_vals, bytes;
 };
 
@@ -928,27 +925,14 @@ md_status hydra_plan(const md_tree* tree, int B, int d, int V, int kmax, HydraPl
   return MD_OK;
 }
 
-// The workspace ranges a heads call needs zero at its start (counters and
-// tickets), as [offset, offset + bytes); bytes = 0 when there are none.
-void heads_zero_range(int M, int d, int V, int K, int kmax, size_t* off, size_t* bytes) {
-  *off = 0;
-  *bytes = 0;
-  // the one-row streaming path's tickets carry a per-call epoch: nothing to clear
-  if (skinny_rows(M)) {
-    const SkinnyPlan pl = skinny_plan(M, d, V, K, kmax);
-    *off = pl.off_tick;
-    *bytes = size_t(K) * (pl.nt1 + pl.nt2) * 4;
-  }
-}
-
 // md_medusa_heads and md_medusa_heads_sampled: checks, then the streaming
 // (one row), weights-as-M (2 .. 32 rows) or row-tile tensor-core path.
 // gumbel_u null: top-k of the logits; else the top-k of the Gumbel keys
-// logit * inv_tau - ln(-ln u). zeroed: heads_zero_range is already zero.
+// logit * inv_tau - ln(-ln u).
 md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv, int32_t M,
                      int32_t d, int32_t V, int32_t K, const int32_t* k_per_head, int32_t kmax, int32_t* topk_ids,
                      float* topk_vals, float* logits_dbg, const float* gumbel_u, float inv_tau, void* ws,
-                     size_t ws_bytes, void* stream, bool zeroed = false) {
+                     size_t ws_bytes, void* stream) {
   if (!h || !W1 || !b1 || !Wv || !k_per_head || !topk_ids || !topk_vals) return MD_ERR_INVALID_ARG;
   md_status s = heads_check(M, d, V, K, kmax);
   if (s != MD_OK) return s;
@@ -966,9 +950,9 @@ md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, con
     if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
     if (pl.NR == 16)
       return launch_heads_skinny<16>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
-                                     logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
+                                     logits_dbg, gumbel_u, inv_tau, w, st);
     return launch_heads_skinny<32>(pl, M, d, V, K, kmax, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals,
-                                   logits_dbg, gumbel_u, inv_tau, w, st, zeroed);
+                                   logits_dbg, gumbel_u, inv_tau, w, st);
   }
   if (!stream_rows(M)) {
     // tensor-core path: h, W1, Wv feed TMA directly (16-byte aligned rows: d % 64, V % 8)
@@ -988,8 +972,7 @@ md_status heads_call(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, con
   const md::heads::Plan pl = md::heads::make_plan(M, d, V, K, kmax, num_sms());
   if (!ws || ws_bytes < pl.bytes || !aligned(ws, 256)) return MD_ERR_WORKSPACE;
   if (M != 1) return MD_ERR_UNSUPPORTED;
-  return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st,
-                         zeroed);
+  return launch_heads<1>(pl, h, W1, b1, Wv, k_per_head, topk_ids, topk_vals, logits_dbg, gumbel_u, inv_tau, w, st);
 }
 
 // Scratch of md_medusa_heads_static: a fixed array in the library's device
@@ -1222,13 +1205,8 @@ md_status md_hydra_draft(const md_tree* tree, const md_bf16* h, int32_t M, const
   uint16_t* x = reinterpret_cast<uint16_t*>(w + p.off_x);
   int32_t* ids = reinterpret_cast<int32_t*>(w + p.off_ids);
   float* vals = reinterpret_cast<float*>(w + p.off_vals);
-  // every level's counters are cleared here, so the levels' kernels follow
-  // one another as dependent launches with no memset between them
-  for (int l = 0; l < p.L; ++l) {
-    size_t zo = 0, zb = 0;
-    heads_zero_range(B * p.n[l], d, V, 1, kmax, &zo, &zb);
-    if (zb && (s = cuda_ok(cudaMemsetAsync(w + p.off_heads[l] + zo, 0, zb, st))) != MD_OK) return s;
-  }
+  // the heads kernels' tickets carry a per-call epoch: nothing is cleared, and
+  // the levels' kernels follow one another as dependent launches
   for (int l = 0; l < p.L; ++l) {
     md::hydra::GatherArgs ga;
     std::memset(&ga, 0, sizeof(ga));
@@ -1249,7 +1227,7 @@ md_status md_hydra_draft(const md_tree* tree, const md_bf16* h, int32_t M, const
     if ((s = heads_call(x, W1 + size_t(l) * d * d, b1 + size_t(l) * d, Wv + size_t(l) * d * V, B * p.n[l], d, V, 1,
                         &tree->kph[l], kmax, ids + r0 * kmax, vals + r0 * kmax,
                         logits_dbg ? logits_dbg + r0 * V : nullptr, nullptr, 1.f, w + p.off_heads[l],
-                        p.heads_bytes[l], stream, true)) != MD_OK)
+                        p.heads_bytes[l], stream)) != MD_OK)
       return s;
   }
   md::hydra::TokenArgs ta;

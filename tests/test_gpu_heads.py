@@ -97,14 +97,16 @@ def test_topk_exact_when_most_candidates_pass_the_threshold(M, K, kk):
     assert np.all(rval[:, :, kk - 1] == 3 * d)
 
 
+@pytest.mark.parametrize("M", [1, 10])
 @pytest.mark.parametrize("fill", ["zeros", "ones", "random"])
-def test_streaming_heads_need_no_cleared_workspace(fill):
-    """The one-row path's tickets carry a per-call epoch: a workspace holding
-    anything at all, and the same workspace reused call after call, give the
-    same results bit for bit (several cut units and split-K tiles)."""
+def test_heads_need_no_cleared_workspace(M, fill):
+    """The tickets of the one-row and weights-as-M paths carry a per-call
+    epoch: a workspace holding anything at all, and the same workspace reused
+    call after call, give the same results bit for bit (cut units and split-K
+    tiles on both paths)."""
     import medusa_draft_heads_b200 as md
-    M, d, V, kph = 1, 1024, 10000, (10, 4, 7, 1)      # 160 units over 148 CTAs: cut units
-    h, W1, b1, Wv = head_weights(77, d, V, len(kph), M)
+    d, V, kph = 1024, 10000, (10, 4, 7, 1)      # one row: 160 units over 148 CTAs, cut units
+    h, W1, b1, Wv = head_weights(77 + M, d, V, len(kph), M)
     ref_ids, ref_vals, ref_log = _run(h, W1, b1, Wv, kph)
     K, kmax = len(kph), max(kph)
     ws = md.workspace(md.heads_workspace_bytes(M, d, V, K, kmax))
