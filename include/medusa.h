@@ -144,7 +144,10 @@ MD_API md_status md_heads_workspace(int32_t M, int32_t d, int32_t V, int32_t K, 
  * topk_ids   [M, K, kmax] int32, topk_vals [M, K, kmax] fp32 (outputs).
  * logits_dbg [M, K, V] fp32 or NULL: when given, the full logits are also
  *            written (debug / parity only; the fused path never needs them).
- * ws, ws_bytes: workspace of at least md_heads_workspace() bytes.
+ * ws, ws_bytes: workspace of at least md_heads_workspace() bytes, any
+ *   contents: nothing in it needs clearing before a call (the kernels'
+ *   arrival tickets carry a per-call epoch), and one workspace serves call
+ *   after call on one stream.
  * Errors: MD_ERR_INVALID_ARG, MD_ERR_UNSUPPORTED, MD_ERR_WORKSPACE, MD_ERR_CUDA. */
 MD_API md_status md_medusa_heads(const md_bf16* h, const md_bf16* W1, const md_bf16* b1, const md_bf16* Wv,
                           int32_t M, int32_t d, int32_t V, int32_t K, const int32_t* k_per_head,
@@ -229,9 +232,8 @@ MD_API md_status md_medusa_heads_sampled(const md_bf16* h, const md_bf16* W1, co
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
  *   first call before any stream capture on the device.
  * - Every call on a device shares the one array and leaves its contents
- *   behind; the call clears what must start at zero itself (the one-row
- *   streaming path needs nothing cleared: its tickets carry a per-call
- *   epoch). Two calls whose
+ *   behind and needs nothing cleared (the heads kernels' tickets carry a
+ *   per-call epoch). Two calls whose
  *   kernels overlap on the GPU (different streams, no ordering between them)
  *   race on the array and give undefined results: order them on one stream
  *   or with events.
