@@ -116,11 +116,12 @@ md_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, 
 }
 
 // The top-k merge is launched in plain stream order: as a dependent launch
-// its CTAs became resident beside the still-running projection kernel and
-// waited there, and the projection ran slower for it (a four-level Hydra
-// draft at 70B shapes took 1.50 ms that way against 1.46 ms in plain order).
-// The kernel's own griddepcontrol instructions are no-ops in this form, and
-// the launch after it can still be a dependent one.
+// (which lets its CTAs start and wait beside the still-running projection)
+// the calls ran slower, although the merge alone is faster (a four-level
+// Hydra draft at 70B shapes took 1.50 ms that way against 1.46 ms in plain
+// order; more shared memory per merge CTA or a later trigger did not change
+// it). The kernel's own griddepcontrol instructions are no-ops in this form,
+// and the launch after it can still be a dependent one.
 inline md_status launch_merge(const md::heads::MergeArgs& ma, int blocks, cudaStream_t st) {
   md::heads::heads_merge_kernel<<<blocks, md::heads::kMergeThreads, 0, st>>>(ma);
   return cuda_ok(cudaGetLastError());
